@@ -1,0 +1,395 @@
+"""Pins of the CPU oracle against things other than itself: closed forms, brute
+force on tiny inputs, library special cases and invariants. CPU only.
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a
+swapped operand, a wrong sign or index, a wrong tie rule) fails it.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import moe_oracle as mo
+
+# ---------------------------------------------------------------- formats
+
+
+def test_e4m3_table_matches_closed_form_landmarks():
+    # OCP E4M3 landmarks: max normal 0x7E = 448, min normal 0x08 = 2^-6,
+    # min subnormal 0x01 = 2^-9, one = 0x38, NaN = 0x7F / 0xFF, -0 = 0x80.
+    t = mo.E4M3_TABLE
+    assert t[0x7E] == 448.0 and t[0xFE] == -448.0
+    assert t[0x08] == 2.0**-6 and t[0x01] == 2.0**-9 and t[0x38] == 1.0
+    assert math.isnan(t[0x7F]) and math.isnan(t[0xFF])
+    assert t[0x80] == 0.0 and math.copysign(1, t[0x80]) == -1
+    assert t[0x07] == 7 * 2.0**-9 and t[0x0F] == 1.875 * 2.0**-6
+
+
+def test_e4m3_table_matches_torch_float8_for_all_codes():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = mo.e4m3_decode(np.arange(256))
+    both_nan = np.isnan(ref) & np.isnan(ours)
+    assert np.all(both_nan | (ref == ours))
+
+
+def test_e4m3_rounding_matches_torch_cast_inside_range():
+    rng = np.random.default_rng(7)
+    v = np.concatenate([rng.normal(0, 1, 20000) * 10.0 ** rng.uniform(-4, 2.6, 20000),
+                        mo.E4M3_TABLE[:126] + 1e-12, (mo.E4M3_TABLE[1:126] + mo.E4M3_TABLE[:125]) / 2])
+    v = v[np.abs(v) <= 448]
+    ours = oracle.round_to_format(v, oracle.E4M3)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    # torch rounds from fp32; compare on inputs that are exact in fp32
+    exact32 = v.astype(np.float32).astype(np.float64) == v
+    assert np.array_equal(ours[exact32], ref[exact32])
+
+
+def test_e4m3_ties_to_even_and_saturation():
+    # 1.0625 lies midway between 1.0 (mantissa 000) and 1.125 (001): even -> 1.0
+    # 1.1875 midway between 1.125 (001) and 1.25 (010): even -> 1.25
+    r = oracle.round_to_format(np.array([1.0625, 1.1875, 449.0, 1e9, -500.0, 2.0**-10, 3 * 2.0**-10, 3 * 2.0**-11]),
+                               oracle.E4M3)
+    assert list(r[:5]) == [1.0, 1.25, 448.0, 448.0, -448.0]
+    assert r[5] == 0.0            # half of min subnormal -> ties to even (0)
+    assert r[6] == 2.0**-9 * 2    # 1.5 min-subnormal -> even (2)
+    assert r[7] == 2.0**-9        # 0.75 min-subnormal -> nearest (1)
+
+
+def test_bf16_and_fp16_rounding_match_torch_from_fp32():
+    rng = np.random.default_rng(3)
+    v = (rng.normal(0, 1, 50000) * 10.0 ** rng.uniform(-30, 30, 50000)).astype(np.float32)
+    v = np.concatenate([v, np.float32([1 + 2**-8, 1 + 3 * 2**-8, -(1 + 2**-8)])])
+    v64 = v.astype(np.float64)
+    ref_b = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.bf16_round(v64), ref_b)
+    vs = v[np.abs(v) < 60000]
+    ref_h = torch.from_numpy(vs).to(torch.float16).to(torch.float64).numpy()
+    assert np.array_equal(mo.fp16_round(vs.astype(np.float64)), ref_h)
+    # ties to even: 1 + 2^-8 -> 1.0 ; 1 + 3*2^-8 -> 1 + 2^-6
+    assert oracle.bf16_round(np.array([1 + 2**-8]))[0] == 1.0
+    assert oracle.bf16_round(np.array([1 + 3 * 2**-8]))[0] == 1 + 2**-6
+
+
+def test_fp32_rounding_is_numpy_float32_cast():
+    rng = np.random.default_rng(5)
+    v = rng.normal(0, 1, 100000) * 10.0 ** rng.uniform(-40, 38, 100000)
+    assert np.array_equal(mo.fp32_round(v), v.astype(np.float32).astype(np.float64))
+
+
+def test_mx_exponent_closed_form_and_shift_invariance():
+    # amax in [2^n, 2^(n+1)) -> X = n - 8 ; zero block -> -127
+    amax = np.array([1.0, 1.999, 2.0, 448.0, 0.75, 2.0**-130, 0.0, 2.0**200])
+    X = oracle.mx_block_exponent(amax)
+    assert list(X) == [-8, -8, -7, 0, -9, -127, -127, 127]
+    rng = np.random.default_rng(11)
+    blk = rng.normal(0, 1, (50, 32))
+    q0 = oracle.quantize_h(blk, "mxfp8")
+    for n in (-5, 3, 17):
+        qn = oracle.quantize_h(blk * 2.0**n, "mxfp8")
+        assert np.array_equal(qn, q0 * 2.0**n)   # 2^n scaling moves X by n only
+
+
+def test_mx_block_max_maps_into_e4m3_range():
+    rng = np.random.default_rng(12)
+    h = rng.normal(0, 3, (8, 64))
+    q = oracle.quantize_h(h, "mxfp8").reshape(8, 2, 32)
+    blk = h.reshape(8, 2, 32)
+    X = oracle.mx_block_exponent(np.abs(blk).max(-1, keepdims=True))
+    codes_vals = q / 2.0**X
+    assert np.all(np.abs(codes_vals) <= 448)
+    assert np.all(np.isin(np.abs(codes_vals), np.abs(mo.E4M3_TABLE[:127])))
+
+
+def test_fp8_row_quant_maps_amax_to_448():
+    rng = np.random.default_rng(2)
+    h = rng.normal(0, 1, (16, 100))
+    q = oracle.quantize_h(h, "fp8")
+    amax = np.abs(h).max(1, keepdims=True)
+    s = mo.fp32_round(amax / 448)
+    i = np.abs(h).argmax(1)
+    np.testing.assert_allclose(np.abs(q[np.arange(16), i]), 448 * s[:, 0], rtol=0)
+    assert np.all(np.isin(np.abs(q / s), np.abs(mo.E4M3_TABLE[:127])))
+    assert np.all(oracle.quantize_h(np.zeros((2, 8)), "fp8") == 0)
+
+
+# ---------------------------------------------------------------- router
+
+
+def _brute_topk(keys, k):
+    """Brute force: the unique k-subset whose every member beats every non-member
+    under (key desc, index asc); returned in that order."""
+    E = len(keys)
+    better = lambda a, b: keys[a] > keys[b] or (keys[a] == keys[b] and a < b)  # noqa: E731
+    for sub in itertools.combinations(range(E), k):
+        rest = [e for e in range(E) if e not in sub]
+        if all(better(a, b) for a in sub for b in rest):
+            return sorted(sub, key=lambda e: (-keys[e], e))
+    raise AssertionError
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_softmax_topk_brute_force_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    E, k = 7, 3
+    logits = rng.integers(-3, 3, (20, E)).astype(np.float32) * 0.5  # many exact ties
+    ids, w = oracle.router_softmax_topk(logits, k, True, 1.0)
+    for t in range(20):
+        assert list(ids[t]) == _brute_topk(list(logits[t]), k)
+        p = np.exp(logits[t].astype(np.float64))
+        ref = p[ids[t]] / p[ids[t]].sum()
+        np.testing.assert_allclose(w[t], ref, rtol=1e-15)
+
+
+def test_softmax_topk_matches_torch_topk_on_distinct_values():
+    rng = np.random.default_rng(9)
+    logits = rng.normal(0, 1, (64, 32)).astype(np.float32)
+    ids, w = oracle.router_softmax_topk(logits, 4, True, 1.0)
+    tv, ti = torch.topk(torch.from_numpy(logits), 4, dim=1)
+    assert np.array_equal(ids, ti.numpy())
+    ref = torch.softmax(tv.double(), dim=1).numpy()
+    np.testing.assert_allclose(w, ref, rtol=1e-14)
+
+
+def test_softmax_no_renorm_is_full_softmax_and_scale_folds():
+    rng = np.random.default_rng(4)
+    logits = rng.normal(0, 2, (10, 16)).astype(np.float32)
+    ids, w = oracle.router_softmax_topk(logits, 5, False, 1.0)
+    full = torch.softmax(torch.from_numpy(logits).double(), 1).numpy()
+    np.testing.assert_allclose(w, np.take_along_axis(full, ids.astype(np.int64), 1), rtol=1e-14)
+    ids2, w2 = oracle.router_softmax_topk(logits, 5, True, 2.5)
+    _, w1 = oracle.router_softmax_topk(logits, 5, True, 1.0)
+    np.testing.assert_allclose(w2.sum(1), 2.5, rtol=1e-14)
+    np.testing.assert_allclose(w2, 2.5 * w1, rtol=1e-15)
+
+
+def test_sigmoid_closed_forms():
+    s = mo.sigmoid_fp32(np.array([0.0, 100.0, -100.0, 2.0, -2.0], np.float32))
+    assert s[0] == 0.5 and s[1] == 1.0
+    assert s[2] == np.float32(1 / (1 + math.exp(100)))
+    assert s[3] == np.float32(1 / (1 + math.exp(-2.0)))
+    assert abs(float(s[3]) + float(s[4]) - 1.0) < 2**-23
+
+
+def _brute_grouped(c, s, k, n_group, topk_group, rsf):
+    E = len(c)
+    gsize = E // n_group
+    groups = [sorted(c[g * gsize:(g + 1) * gsize], reverse=True) for g in range(n_group)]
+    score = [np.float32(gr[0]) + np.float32(gr[1]) if gsize > 1 else np.float32(gr[0]) for gr in groups]
+    kept = _brute_topk([float(x) for x in score], topk_group)
+    allowed = [e for e in range(E) if e // gsize in kept]
+    sel = sorted(allowed, key=lambda e: (-c[e], e))[:k]
+    ws = np.array([float(s[e]) for e in sel])
+    return sel, ws / ws.sum() * rsf
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_grouped_sigmoid_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    E, n_group, topk_group, k = 12, 4, 2, 3
+    logits = (rng.integers(-4, 4, (16, E)) * 0.25).astype(np.float32)   # ties in c and groups
+    bias = (rng.integers(-2, 2, E) * 0.125).astype(np.float32)
+    ids, w = oracle.router_grouped_sigmoid_topk(logits, bias, k, n_group, topk_group, True, 2.5)
+    s = mo.sigmoid_fp32(logits).astype(np.float32)
+    for t in range(16):
+        c = [float(np.float32(s[t, e] + bias[e])) for e in range(E)]
+        sel, ref = _brute_grouped(c, s[t], k, n_group, topk_group, 2.5)
+        assert list(ids[t]) == sel
+        np.testing.assert_allclose(w[t], ref, rtol=1e-15)
+
+
+def test_grouped_reduces_to_plain_sigmoid_topk():
+    # one group, or all groups kept: plain top-k of c; zero bias: top-k of the
+    # logits themselves (sigmoid is increasing; distinct logits far apart)
+    rng = np.random.default_rng(21)
+    logits = rng.normal(0, 1, (32, 16)).astype(np.float32)
+    ref_ids, _ = oracle.router_softmax_topk(logits, 4, True, 1.0)
+    for n_group, topk_group in ((1, 1), (4, 4), (16, 16)):
+        ids, w = oracle.router_grouped_sigmoid_topk(logits, None, 4, n_group, topk_group, True, 1.0)
+        assert np.array_equal(ids, ref_ids)
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+
+
+def test_grouped_all_experts_selected_weights_are_normalised_scores():
+    rng = np.random.default_rng(22)
+    logits = rng.normal(0, 1, (5, 8)).astype(np.float32)
+    ids, w = oracle.router_grouped_sigmoid_topk(logits, None, 8, 2, 2, True, 1.0)
+    s = mo.sigmoid_fp32(logits)
+    for t in range(5):
+        assert sorted(ids[t]) == list(range(8))
+        np.testing.assert_allclose(w[t], s[t, ids[t]] / s[t].sum(), rtol=1e-15)
+
+
+# ---------------------------------------------------------------- sort
+
+
+@pytest.mark.parametrize("T,k,E,bm", [(16, 2, 8, 16), (37, 3, 5, 4), (1, 1, 1, 8), (64, 8, 128, 16), (50, 6, 64, 128)])
+def test_align_sort_matches_library_stable_sort(T, k, E, bm):
+    rng = np.random.default_rng(T * 7 + E)
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]) if k <= E else None
+    r = oracle.align_sort(ids, E, bm)
+    flat = ids.reshape(-1)
+    order = np.argsort(flat, kind="stable")          # library stable sort
+    real = r["sorted_ids"][r["sorted_ids"] != T * k]
+    assert np.array_equal(real, order)
+    assert np.array_equal(r["expert_counts"], np.bincount(flat, minlength=E))
+    # invariants: every flat slot once, segments aligned to bm, single-expert blocks
+    assert r["expert_counts"].sum() == T * k
+    assert np.all(np.diff(r["expert_offsets"]) % bm == 0)
+    assert r["num_padded"] == len(r["sorted_ids"]) <= oracle.sorted_capacity(T, k, E, bm)
+    for b, e in enumerate(r["block_expert"]):
+        blk = r["sorted_ids"][b * bm:(b + 1) * bm]
+        assert np.all((blk == T * k) | (flat[np.minimum(blk, T * k - 1)] == e))
+        assert r["expert_offsets"][e] <= b * bm < r["expert_offsets"][e + 1]
+    tokens_seen = np.bincount(real // k, minlength=T)
+    assert np.all(tokens_seen == k)  # each token sits in exactly k expert slots
+
+
+# ---------------------------------------------------------------- gate
+
+
+def test_gate_closed_form():
+    K = 64
+    x = np.ones((3, K))
+    w = np.array([0.0, 1 / 64, -2 / 64])[:, None] * np.ones((1, K))
+    for i, c in enumerate([0.0, 1.0, -2.0]):
+        g = oracle.shared_gate(x[i:i + 1], w[i], True, oracle.BF16)
+        assert g[0] == oracle.bf16_round(1 / (1 + math.exp(-c)))
+    assert oracle.shared_gate(x[:1], w[0], True, oracle.BF16)[0] == 0.5
+    g = oracle.shared_gate(x[:1], w[1] * 3, False, oracle.FP16)
+    assert g[0] == 3.0
+
+
+def test_gate_brute_force_dot():
+    rng = np.random.default_rng(8)
+    x = rng.normal(0, 1, (4, 33))
+    w = rng.normal(0, 0.02, 33)
+    g = oracle.shared_gate(x, w, True, oracle.FP16)
+    for t in range(4):
+        d = sum(x[t, i] * w[i] for i in range(33))
+        assert g[t] == mo.fp16_round(1 / (1 + math.exp(-d)))
+
+
+# ---------------------------------------------------------------- expert / layer
+
+
+def test_silu_closed_form():
+    z = np.array([0.0, 1.0, -1.0, 20.0])
+    np.testing.assert_allclose(oracle.silu(z), [0.0, 1 / (1 + math.exp(-1)), -1 / (1 + math.exp(1)),
+                                                20 / (1 + math.exp(-20))], rtol=1e-15)
+
+
+def test_expert_forward_brute_force_loops():
+    """Tiny expert written out with scalar loops: catches a transposed W13/W2,
+    swapped gate/up halves, a missing SiLU or a scale in the wrong place."""
+    rng = np.random.default_rng(31)
+    H, I = 5, 3
+    x = rng.normal(0, 1, H)
+    w13 = rng.normal(0, 1, (2 * I, H))
+    w2 = rng.normal(0, 1, (H, I))
+    sx, s13, s2 = 0.5, 0.25, 3.0
+    y = oracle.expert_forward(x, w13, w2, I, "fp8", sx, s13, s2)
+    a = [sum(w13[r, c] * x[c] for c in range(H)) * sx * s13 for r in range(2 * I)]
+    h = [a[i] / (1 + math.exp(-a[i])) * a[I + i] for i in range(I)]
+    amax = max(abs(v) for v in h)
+    s = float(np.float32(amax / 448))
+    hq = [float(oracle.round_to_format(np.array([v / s]), oracle.E4M3)[0]) * s for v in h]
+    ref = [sum(w2[o, i] * hq[i] for i in range(I)) * s2 for o in range(H)]
+    np.testing.assert_allclose(y, ref, rtol=1e-13)
+
+
+def test_expert_forward_identity_weights_closed_form():
+    # W13 = [I; I] (gate = up = identity), W2 = identity: y = bf16(silu(x) * x)
+    n = 8
+    x = np.linspace(-3, 3, n)
+    w13 = np.vstack([np.eye(n), np.eye(n)])
+    y = oracle.expert_forward(x, w13, np.eye(n), n, "bf16")
+    assert np.array_equal(y, oracle.bf16_round(x * x / (1 + np.exp(-x))))
+
+
+def _tiny_cfg(**kw):
+    cfg = dict(T=6, H=32, E=4, top_k=2, I=32, Is=32, dtype="bf16", route="softmax", n_group=1,
+               topk_group=1, rsf=1.0, renormalize=True, shared_gate=True)
+    cfg.update(kw)
+    return cfg
+
+
+def _tiny_inputs(cfg, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    T, H, E, I, Is = (cfg[n] for n in ("T", "H", "E", "I", "Is"))
+    r = lambda *s, sd=1.0: (torch.randn(*s, generator=g) * sd)  # noqa: E731
+    return {"logits": r(T, E), "x": r(T, H).bfloat16(), "w_gate": r(H, sd=0.1).bfloat16(),
+            "w13": r(E, 2 * I, H, sd=0.1).bfloat16(), "w2": r(E, H, I, sd=0.1).bfloat16(),
+            "w13s": r(2 * Is, H, sd=0.1).bfloat16(), "w2s": r(H, Is, sd=0.1).bfloat16(),
+            "correction_bias": None}
+
+
+def test_layer_brute_force_tiny():
+    cfg = _tiny_cfg()
+    inp = _tiny_inputs(cfg)
+    r = oracle.moe_layer(cfg, inp)
+    x = inp["x"].double().numpy()
+    lg = inp["logits"].numpy()
+    for t in range(cfg["T"]):
+        order = sorted(range(cfg["E"]), key=lambda e: (-lg[t, e], e))[:2]
+        p = [math.exp(float(lg[t, e]) - float(lg[t, order[0]])) for e in order]
+        wts = [v / sum(p) for v in p]
+        d = sum(x[t, h] * float(inp["w_gate"][h]) for h in range(cfg["H"]))
+        gate = float(oracle.bf16_round(np.array([1 / (1 + math.exp(-d))]))[0])
+
+        def mlp(w13, w2, I):
+            w13 = w13.double().numpy()
+            w2 = w2.double().numpy()
+            a = [sum(w13[i, c] * x[t, c] for c in range(cfg["H"])) for i in range(2 * I)]
+            h = oracle.bf16_round(np.array([a[i] / (1 + math.exp(-a[i])) * a[I + i] for i in range(I)]))
+            return np.array([sum(w2[o, i] * h[i] for i in range(I)) for o in range(cfg["H"])])
+        addend = oracle.bf16_round(gate * mlp(inp["w13s"], inp["w2s"], cfg["Is"]))
+        routed = sum(wts[j] * mlp(inp["w13"][order[j]], inp["w2"][order[j]], cfg["I"]) for j in range(2))
+        ref = oracle.bf16_round(addend + routed)
+        assert list(r["topk_ids"][t]) == order
+        # brute force and oracle differ only in float64 summation order
+        assert np.max(np.abs(r["out"][t] - ref)) <= 2.0**-8 * np.max(np.abs(ref)) + 1e-12
+
+
+def test_layer_invariants_fold_and_addend():
+    cfg = _tiny_cfg(shared_gate=False)
+    inp = _tiny_inputs(cfg, seed=1)
+    base = oracle.moe_layer(cfg, inp)
+    scaled = oracle.moe_layer(dict(cfg, rsf=2.5), inp)
+    # folding the scale into the weights == scaling the routed output
+    np.testing.assert_allclose(scaled["routed"], 2.5 * base["routed"], rtol=1e-12, atol=1e-15)
+    # shared expert with zero weights: the output is the routed sum alone
+    zero = dict(inp, w2s=torch.zeros_like(inp["w2s"]))
+    rz = oracle.moe_layer(cfg, zero)
+    assert np.all(rz["addend"] == 0)
+    np.testing.assert_array_equal(rz["out"], oracle.bf16_round(rz["routed"]))
+    # the addend path equals a separate add of the two bf16-free parts
+    np.testing.assert_array_equal(base["out"], oracle.bf16_round(base["addend"] + base["routed"]))
+
+
+def test_layer_equal_logits_give_uniform_weights():
+    cfg = _tiny_cfg(E=4, top_k=4, shared_gate=False)
+    inp = _tiny_inputs(cfg, seed=2)
+    inp["logits"] = torch.zeros(cfg["T"], 4)
+    r = oracle.moe_layer(cfg, inp)
+    assert np.all(r["topk_ids"] == np.arange(4))
+    np.testing.assert_allclose(r["topk_weights"], 0.25, rtol=0)
+
+
+def test_layer_single_expert_is_dense_mlp():
+    """E = 1, k = 1: the routed part is one dense MLP (checked with torch
+    matmuls in float64 on the decoded weights)."""
+    cfg = _tiny_cfg(E=1, top_k=1, shared_gate=False)
+    inp = _tiny_inputs(cfg, seed=3)
+    r = oracle.moe_layer(cfg, inp)
+    x = inp["x"].double()
+    w13 = inp["w13"][0].double()
+    a = x @ w13.T
+    h = torch.nn.functional.silu(a[:, :32]) * a[:, 32:]
+    h = torch.from_numpy(oracle.bf16_round(h.numpy()))
+    y = h @ inp["w2"][0].double().T
+    np.testing.assert_allclose(r["routed"], y.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(r["topk_weights"], 1.0)
