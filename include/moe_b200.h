@@ -1,0 +1,234 @@
+/*
+ * moe_b200.h - C ABI of the B200 (sm_100a) routed + shared-expert MoE layer.
+ *
+ * One MoE layer forward = five calls, in this order on the caller's streams:
+ *
+ *   main stream:  moe_router_topk -> moe_align_sort -> moe_stage1_gemm
+ *                 -> moe_stage2_gemm_accumulate (waits on the addend event)
+ *   side stream:  shared_expert_gate_dot -> moe_stage1_gemm (identity routing)
+ *                 -> moe_stage2_gemm_accumulate (identity routing, writes the
+ *                    addend) -> record the addend event
+ *
+ * Sources (web pages; the section named is where the operation is stated):
+ *   [65207] vllm-project/vllm PR 65207, "Purpose": commit 1 folds
+ *           routed_scaling_factor into the top-k weights inside
+ *           biased_grouped_topk; commit 2 hands the shared-expert output to the
+ *           routed experts as the stage-2 addend plus a ready event, the
+ *           aux-stream shared expert overlapping sorting and stage 1, the
+ *           stage-2 GEMM epilogue accumulating it; "Dependencies": the
+ *           capability is feature-detected (supports_output_addend).
+ *           Reviewer measurements, "Commits 2 and 3": moe_sorting without
+ *           zeroing the output.
+ *   [6106]  ROCm/aiter PR 6106 "[Triton/Gluon] Add per token scale to a8w8 moe
+ *           gemm", "Technical Details": x_token_scale (fp32, one per row of x)
+ *           and w_expt_scale (fp32, one per expert) multiply the fp32
+ *           accumulator in the epilogue before activation and fused quant;
+ *           rows follow the gather index; MXFP8 uses BLOCK_K = 32, K % 32 == 0.
+ *   [56789] vllm-project/vllm PR 56789 (shared_expert_gate as a tiny dot),
+ *           "Summary" and "Commits": sigmoid(x . w_gate) as one fp32-
+ *           accumulated dot with the sigmoid folded in; the output is stored in
+ *           the input dtype so the store does the rounding.
+ *
+ * Conventions, all calls:
+ *   - Tensor pointers are DEVICE pointers owned by the caller. The calls
+ *     allocate no memory. Every call is asynchronous on the given stream.
+ *   - Arguments are checked on the host first; on any invalid argument the
+ *     call returns a negative status and launches nothing.
+ *   - MOE_ERR_CUDA: a CUDA runtime call failed; moe_last_cuda_error() gives
+ *     the message (per thread).
+ *   - Kernels never trap: a device-side check or a bounded wait that gives up
+ *     records a code in a device error word read by moe_device_error().
+ *   - Layouts are row-major and dense unless stated. T tokens, H hidden, E
+ *     routed experts, k = top_k, I expert intermediate size.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* CUDA handles are passed as opaque pointers (cudaStream_t / cudaEvent_t). */
+typedef void* moe_stream_t;
+typedef void* moe_event_t;
+
+typedef int moe_status_t;
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)       /* null pointer, out-of-range size or mode */
+#define MOE_ERR_UNSUPPORTED_DTYPE (-2) /* dtype not accepted by this call */
+#define MOE_ERR_ALIGNMENT (-3)         /* pointer not 16-byte aligned, K % 32 != 0 for MXFP8 */
+#define MOE_ERR_SHAPE (-4)             /* sizes the kernels do not cover */
+#define MOE_ERR_CUDA (-5)              /* a CUDA runtime / driver call failed */
+#define MOE_ERR_DEVICE (-6)            /* device error word was set (moe_device_error) */
+
+/* Operand formats. */
+#define MOE_DT_BF16 0
+#define MOE_DT_FP16 1
+#define MOE_DT_FP8_E4M3 2   /* e4m3 codes; fp32 scale per token row of x, per expert of W [6106] */
+#define MOE_DT_MXFP8_E4M3 3 /* e4m3 codes; ue8m0 byte per 32 K elements of every row [6106] */
+#define MOE_DT_F32 4
+
+/* Routing modes of moe_router_topk. */
+#define MOE_ROUTE_SOFTMAX 0
+#define MOE_ROUTE_GROUPED_SIGMOID 1
+
+/* Largest sizes the kernels cover. */
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 32
+
+/* ------------------------------------------------------------------------ */
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t status);
+/* Library version string. */
+const char* moe_version(void);
+/* Message of the last failed CUDA call made by this thread inside the library. */
+const char* moe_last_cuda_error(void);
+/* 1: moe_stage2_gemm_accumulate accepts an output addend and a ready event
+ * (the capability query of [65207] "Dependencies"). */
+int moe_supports_output_addend(void);
+
+/* Reads the current device's error word into *code (0 = none) and clears it.
+ * Synchronises `stream` first. Codes: 1 = bounded mbarrier wait gave up,
+ * 2 = expert id out of range in the sort, 3 = sorted slot id out of range. */
+moe_status_t moe_device_error(int* code, moe_stream_t stream);
+
+/* Number of int32 slots the padded sort output may need: T*top_k +
+ * E*(block_m - 1) rounded up to a multiple of block_m ("capacity rows").
+ * sorted_ids holds this many entries, block_expert this / block_m, and the
+ * stage-1 output h this many rows. */
+size_t moe_sorted_capacity(int T, int top_k, int E, int block_m);
+
+/* Bytes of the fp32 accumulation workspace of moe_stage2_gemm_accumulate:
+ * T*H floats followed by T*ceil(H/128) int32 arrival counters. The caller
+ * zeroes it ONCE after allocating it; each complete call leaves it zeroed. */
+size_t moe_stage2_workspace_bytes(int T, int H);
+
+/* Bytes of the per-row partial-amax buffer that moe_stage1_gemm writes for
+ * MOE_DT_FP8_E4M3 (ceil(I/64) floats per sorted row); 0 for other dtypes. */
+size_t moe_stage1_amax_bytes(int dtype, int rows, int I);
+
+/* ------------------------------------------------------------------------ */
+
+/* moe_router_topk: top-k routing of T tokens over E experts.
+ * [65207] "Purpose", commit 1: routed_scaling_factor is applied inside this
+ * call, to the top-k weights, instead of to the layer output.
+ *
+ *   logits          fp32 [T,E]   router logits (the model's gate linear).
+ *   correction_bias fp32 [E] or NULL (GROUPED_SIGMOID only; NULL = 0).
+ *   mode MOE_ROUTE_SOFTMAX: pick the k largest logits (ties: lower index);
+ *        weights exp(l_j - m)/sum_sel exp(l_i - m) (renormalize != 0) or the
+ *        full softmax at the picked experts (renormalize == 0).
+ *   mode MOE_ROUTE_GROUPED_SIGMOID: s = fp32(sigmoid(l)) evaluated in double;
+ *        c = s + bias (fp32); group score = sum of the two largest c of each
+ *        of n_group equal groups; keep topk_group groups (ties: lower group);
+ *        pick k experts of the kept groups by c (ties: lower index); weights
+ *        s_j / sum_sel s (renormalize != 0) or s_j.
+ *   Both modes multiply the weights by routed_scaling_factor.
+ *   topk_ids     int32 [T,k]  experts in selection order (best first).
+ *   topk_weights fp32  [T,k]  same order.
+ * Checks: 1 <= T, 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= min(E, MOE_MAX_TOPK);
+ * grouped mode: n_group divides E, 1 <= topk_group <= n_group <= 32,
+ * k <= topk_group * E / n_group. */
+moe_status_t moe_router_topk(const float* logits, const float* correction_bias, int T, int E,
+                             int top_k, int mode, int n_group, int topk_group, int renormalize,
+                             float routed_scaling_factor, int32_t* topk_ids, float* topk_weights,
+                             moe_stream_t stream);
+
+/* moe_align_sort: group the T*k routed slots by expert for the grouped GEMMs
+ * ([65207] reviewer measurements: moe_sorting; here it never zeroes the layer
+ * output - the stage-2 epilogue owns the output; [6106]: the GEMM rows follow
+ * this gather index).
+ *   topk_ids      int32 [T,k]; slot f = t*k + j.
+ *   sorted_ids    int32 [>= moe_sorted_capacity]: experts in order 0..E-1;
+ *                 inside an expert ascending f (stable); every expert segment
+ *                 padded to a multiple of block_m with the sentinel T*k.
+ *                 Entries at and past *num_padded are not written.
+ *   block_expert  int32 [>= capacity/block_m]: owning expert of each block.
+ *   expert_counts int32 [E]; expert_offsets int32 [E+1] (padded prefix sum);
+ *   num_padded    int32 [1] = expert_offsets[E].
+ * Checks: block_m in {16,32,64,128,256}; T*k <= 1<<20; E <= MOE_MAX_EXPERTS.
+ * An expert id outside [0,E) sets device error 2 and is dropped. */
+moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
+                            int32_t* sorted_ids, int32_t* block_expert, int32_t* expert_counts,
+                            int32_t* expert_offsets, int32_t* num_padded, moe_stream_t stream);
+
+/* moe_stage1_gemm: per sorted row r (slot f = sorted_ids[r], token t = f/k,
+ * expert e = block_expert[r/block_m]):
+ *     a   = W13[e] . x[t]                           (2I outputs, fp32 accumulate)
+ *     a  *= x_scale[t] * w13_scale[e]               (MOE_DT_FP8_E4M3; [6106])
+ *     h_r = SiLU(a[0:I]) * a[I:2I]
+ * tcgen05 tensor cores, weights streamed by TMA, token rows gathered by TMA.
+ *   dtype      MOE_DT_BF16 or MOE_DT_FP8_E4M3.
+ *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8) or NULL.
+ *   w13        [E,2I,H]: rows 0..I-1 gate, I..2I-1 up (K = H contiguous);
+ *              w13_scale fp32 [E] (FP8) or NULL.
+ *   sorted_ids / block_expert / num_padded: from moe_align_sort with the same
+ *              block_m. sorted_ids == NULL selects identity routing (row r =
+ *              token r, expert 0, rows padded to a multiple of block_m; used
+ *              for the shared expert, E = 1, k = 1); block_expert and
+ *              num_padded are then ignored.
+ *   h          [capacity rows, I] bf16 (padded rows hold don't-care values).
+ *              BF16: the stage-2 operand. FP8: the unquantised h; the e4m3
+ *              quantisation (one scale amax/448 per row, [6106] "fused quant")
+ *              happens when stage 2 stages the rows for the tensor core.
+ *   h_amax     fp32 [ceil(I/64), capacity rows]: FP8 per-tile row amax (NULL
+ *              for BF16).
+ * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8), I % 64 == 0, block_m in
+ * {16,32,64,128,256}, 16-byte aligned x, w13, h. */
+moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, const void* w13,
+                             const float* w13_scale, const int32_t* sorted_ids,
+                             const int32_t* block_expert, const int32_t* num_padded, int T,
+                             int top_k, int H, int I, int E, int block_m, void* h, float* h_amax,
+                             moe_stream_t stream);
+
+/* moe_stage2_gemm_accumulate: per sorted row r (slot f, token t, expert e):
+ *     y_r   = W2[e] . h_r                           (H outputs, fp32 accumulate)
+ *     y_r  *= h_scale_r * w2_scale[e]               (MOE_DT_FP8_E4M3; [6106])
+ *     out[t] = bf16( addend[t] + sum over the k slots of t of weight[f] * y_r )
+ * The top-k weight, the scatter-reduce over the k slots of a token and the
+ * shared-expert addend all happen in this GEMM's epilogue ([65207] "Purpose",
+ * commit 2): no separate scale, add or zeroing kernel runs. Partial sums meet
+ * in an fp32 workspace; the epilogue that brings a token's last slot adds the
+ * addend, rounds once to bf16, writes out and re-zeroes its workspace slice.
+ *   dtype       as stage 1; h / h_amax are stage 1's outputs.
+ *   w2          [E,H,I] (K = I contiguous); w2_scale fp32 [E] (FP8) or NULL.
+ *   weights     [T*k] per slot f (routing weights, scale folded in), dtype
+ *               weights_dtype = MOE_DT_F32, or MOE_DT_BF16 / MOE_DT_FP16 (the
+ *               shared gate's output); NULL = 1.0.
+ *   addend      bf16 [T,H] or NULL. addend_ready: event recorded after the
+ *               addend was written, or NULL; the call makes `stream` wait on it
+ *               right before the GEMM ([65207]: only right before stage 2).
+ *               addend may equal out (in-place accumulate).
+ *   acc_ws      moe_stage2_workspace_bytes(T,H) bytes, zeroed once by the
+ *               caller; unused (may be NULL) when top_k == 1.
+ *   out         bf16 [T,H]; every token row is written exactly once.
+ * Identity routing (sorted_ids == NULL): as in stage 1; with top_k == 1 each
+ * row's result goes straight to out (this is how the shared expert's output
+ * becomes the addend of the routed call).
+ * Checks: H % 16 == 0, I % 64 == 0 (bf16) / % 128 == 0 (fp8), block_m as
+ * stage 1, 16-byte aligned h, w2, out, addend. */
+moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h_amax,
+                                        const void* w2, const float* w2_scale, const void* weights,
+                                        int weights_dtype, const int32_t* sorted_ids,
+                                        const int32_t* block_expert, const int32_t* num_padded,
+                                        int T, int top_k, int H, int I, int E, int block_m,
+                                        const void* addend, moe_event_t addend_ready, void* acc_ws,
+                                        void* out, moe_stream_t stream);
+
+/* shared_expert_gate_dot: out[t] = sigmoid(sum_k x[t,k] * w[k]) ([56789]),
+ * one fused kernel, fp32 accumulation, the result stored in x's dtype (the
+ * store rounds). apply_sigmoid == 0 stores the plain dot.
+ *   dtype MOE_DT_BF16 or MOE_DT_FP16 (x, w and out share it).
+ *   x [T,K], w [K], out [T]. Checks: T >= 1, K >= 1. */
+moe_status_t shared_expert_gate_dot(int dtype, const void* x, const void* w, int T, int K,
+                                    int apply_sigmoid, void* out, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -368,19 +368,22 @@ def quantize_h(h, mode: str) -> np.ndarray:
     raise ValueError(mode)
 
 
-def expert_forward(x_t, w13, w2, I: int, hmode: str, s_x=1.0, s_w13=1.0, s_w2=1.0):
-    """One expert on one token (float64), in the order the pages give:
-
+def expert_hidden(x_t, w13, I: int, s_x=1.0, s_w13=1.0):
+    """Stage-1 value of one expert on one token, before quantisation:
     acc1 = W13 @ x (2I outputs); a = acc1 * s_x * s_w13 (scales on the fp32
-    accumulator before the activation); h = SiLU(a[:I]) * a[I:]; h is quantised
-    (``quantize_h``); y = (W2 @ h) * s_w2, where a per-row scale of h is already
-    inside the dequantised h. MX block scales are inside the decoded operands.
-    Returns y [H].
-    """
+    accumulator before the activation); h = SiLU(a[:I]) * a[I:]."""
     acc1 = np.asarray(w13, np.float64) @ np.asarray(x_t, np.float64)
     a = acc1 * s_x * s_w13
-    h = silu(a[:I]) * a[I:]
-    hq = quantize_h(h, hmode)
+    return silu(a[:I]) * a[I:]
+
+
+def expert_forward(x_t, w13, w2, I: int, hmode: str, s_x=1.0, s_w13=1.0, s_w2=1.0):
+    """One expert on one token (float64), in the order the pages give:
+    h = ``expert_hidden``; h is quantised (``quantize_h``); y = (W2 @ h) * s_w2,
+    where a per-row scale of h is already inside the dequantised h. MX block
+    scales are inside the decoded operands. Returns y [H].
+    """
+    hq = quantize_h(expert_hidden(x_t, w13, I, s_x, s_w13), hmode)
     return (np.asarray(w2, np.float64) @ hq) * s_w2
 
 

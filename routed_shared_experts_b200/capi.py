@@ -1,0 +1,150 @@
+"""ctypes binding of ``libmoe_b200.so`` (C ABI in ``include/moe_b200.h``).
+
+Argument marshalling only: each function takes torch tensors (device memory)
+and plain numbers, checks device and contiguity, and calls the C entry point of
+the same name on the current (or given) CUDA stream. A non-zero status raises
+``MoEError``. There is no fallback: if the library is not built, the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+MOE_OK = 0
+MOE_DT_BF16, MOE_DT_FP16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3, MOE_DT_F32 = 0, 1, 2, 3, 4
+MOE_ROUTE_SOFTMAX, MOE_ROUTE_GROUPED_SIGMOID = 0, 1
+DTYPES = {"bf16": MOE_DT_BF16, "fp16": MOE_DT_FP16, "fp8": MOE_DT_FP8_E4M3, "mxfp8": MOE_DT_MXFP8_E4M3,
+          "f32": MOE_DT_F32}
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+# name -> (restype, argtypes)
+_P, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_version": (ctypes.c_char_p, []),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
+    "moe_supports_output_addend": (_I, []),
+    "moe_device_error": (_I, [ctypes.POINTER(ctypes.c_int), _P]),
+    "moe_sorted_capacity": (_SZ, [_I, _I, _I, _I]),
+    "moe_stage2_workspace_bytes": (_SZ, [_I, _I]),
+    "moe_stage1_amax_bytes": (_SZ, [_I, _I, _I]),
+    "moe_router_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "moe_align_sort": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_stage2_gemm_accumulate": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                        _P, _P, _P]),
+    "shared_expert_gate_dot": (_I, [_I, _P, _P, _I, _I, _I, _P, _P]),
+}
+
+_LIB = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        lib_ = lib()
+        msg = lib_.moe_status_string(status).decode()
+        cuda = lib_.moe_last_cuda_error().decode()
+        super().__init__(f"{fn}: {msg}" + (f" ({cuda})" if status == -5 and cuda else ""))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once). Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m routed_shared_experts_b200.build")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = handle
+    return _LIB
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor or None")
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _event(ev):
+    if ev is None:
+        return None
+    return ev.cuda_event or None
+
+
+def _check(name: str, status: int):
+    if status != MOE_OK:
+        raise MoEError(name, status)
+
+
+def sorted_capacity(T: int, top_k: int, E: int, block_m: int) -> int:
+    return lib().moe_sorted_capacity(T, top_k, E, block_m)
+
+
+def stage2_workspace_bytes(T: int, H: int) -> int:
+    return lib().moe_stage2_workspace_bytes(T, H)
+
+
+def stage1_amax_bytes(dtype: int, rows: int, I: int) -> int:
+    return lib().moe_stage1_amax_bytes(dtype, rows, I)
+
+
+def device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("moe_device_error", lib().moe_device_error(ctypes.byref(code), _stream(stream)))
+    return code.value
+
+
+def moe_router_topk(logits, correction_bias, top_k, mode, n_group, topk_group, renormalize,
+                    routed_scaling_factor, topk_ids, topk_weights, stream=None):
+    T, E = logits.shape
+    _check("moe_router_topk", lib().moe_router_topk(
+        _ptr(logits), _ptr(correction_bias), T, E, top_k, mode, n_group, topk_group, int(renormalize),
+        float(routed_scaling_factor), _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+
+
+def moe_align_sort(topk_ids, E, block_m, sorted_ids, block_expert, expert_counts, expert_offsets, num_padded,
+                   stream=None):
+    T, k = topk_ids.shape
+    _check("moe_align_sort", lib().moe_align_sort(
+        _ptr(topk_ids), T, k, E, block_m, _ptr(sorted_ids), _ptr(block_expert), _ptr(expert_counts),
+        _ptr(expert_offsets), _ptr(num_padded), _stream(stream)))
+
+
+def moe_stage1_gemm(dtype, x, x_scale, w13, w13_scale, sorted_ids, block_expert, num_padded, T, top_k, H, I, E,
+                    block_m, h, h_amax, stream=None):
+    _check("moe_stage1_gemm", lib().moe_stage1_gemm(
+        dtype, _ptr(x), _ptr(x_scale), _ptr(w13), _ptr(w13_scale), _ptr(sorted_ids), _ptr(block_expert),
+        _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(h), _ptr(h_amax), _stream(stream)))
+
+
+def moe_stage2_gemm_accumulate(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids, block_expert,
+                               num_padded, T, top_k, H, I, E, block_m, addend, addend_ready, acc_ws, out,
+                               stream=None):
+    _check("moe_stage2_gemm_accumulate", lib().moe_stage2_gemm_accumulate(
+        dtype, _ptr(h), _ptr(h_amax), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
+        _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
+        _event(addend_ready), _ptr(acc_ws), _ptr(out), _stream(stream)))
+
+
+def shared_expert_gate_dot(dtype, x, w, apply_sigmoid, out, stream=None):
+    T, K = x.shape
+    _check("shared_expert_gate_dot", lib().shared_expert_gate_dot(
+        dtype, _ptr(x), _ptr(w), T, K, int(apply_sigmoid), _ptr(out), _stream(stream)))

@@ -1,0 +1,428 @@
+// gemm.cuh - grouped GEMMs of the MoE layer on tcgen05 tensor cores.
+//
+// Stage 1 (gate_up + SiLU-and-mul) and stage 2 (down + weighted scatter-reduce
+// + shared-expert addend) share one persistent, warp-specialised kernel:
+//
+//   warp 0      TMA producer: weight tile (128 rows x 128 K-bytes) and token
+//               tile (BN rows x 128 K-bytes) per pipeline stage. Stage-1 token
+//               rows are gathered from x by TMA gather4 through sorted_ids.
+//   warp 1      TMEM allocator + MMA issuer (one thread): tcgen05.mma with the
+//               weights as A (M = 128) and the tokens as B (N = BN), fp32
+//               accumulator in TMEM, double-buffered across tiles.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator, then
+//               stage 1: optional fp8 scales, SiLU(gate) * up, store h;
+//               stage 2: scales x top-k weight, fp32 red.add into the token
+//               row, and the CTA that brings a token's last slot adds the
+//               addend, rounds once to bf16, writes out and re-zeroes.
+//
+// Weights on the MMA M side ("swap AB") keep the 128-row MMA fully used even
+// when an expert holds a handful of tokens (decode), so the kernel streams
+// weights at the rate the pipeline depth allows.
+//
+// Sources: vllm-project/vllm PR 65207 "Purpose" (commit 2: the shared-expert
+// output is the stage-2 addend, accumulated in the GEMM2 epilogue; commit 1:
+// the routed scale is already inside the top-k weights); ROCm/aiter PR 6106
+// "Technical Details" (per-row activation scale x per-expert weight scale on
+// the fp32 accumulator, before activation; rows follow the gather index).
+#pragma once
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kGemmThreads = 192;
+constexpr int kTileM = 128;       // weight rows per tile = MMA M
+constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte swizzle row
+constexpr int kEpiThreads = 128;
+constexpr int kEpiBar = 1;        // named barrier of the 4 epilogue warps
+
+struct GemmArgs {
+  const int32_t* sorted_ids;  // nullptr: identity routing (row r = token r, expert 0)
+  const int32_t* block_expert;
+  const int32_t* num_padded;
+  int identity_rows;  // identity routing: rows padded to BN
+  int cap_blocks;     // token blocks the sorted buffers can hold
+  int T, top_k, H, I;
+  int n_mt;    // weight tiles per token block
+  int num_kb;  // K stages per tile
+  // stage 1 outputs
+  __nv_bfloat16* h;  // [rows, I]
+  float* h_amax;     // fp8: [ceil(I/64)][rows_cap]
+  int rows_cap;
+  const float* x_scale;  // fp8: [T]
+  const float* w_scale;  // fp8: [E]
+  // stage 2
+  const float* h_amax_in;  // fp8: stage-1 partial amax
+  int n_amax_tiles;
+  const void* weights;  // [T*k] or nullptr
+  int weights_dtype;    // 4 = f32, 0 = bf16, 1 = fp16
+  const __nv_bfloat16* addend;
+  float* ws;
+  int* counters;
+  __nv_bfloat16* out;
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr int kABytes = kTileM * kTileKBytes;
+  static constexpr int kBBytes = BN * kTileKBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
+  // tmem slot, abort flag, ok flag, pad, rows[BN], last[BN], amax_part[4][BN]
+  static constexpr int kMiscBytes = 16 + BN * 4 + BN * 4 + 4 * BN * 4;
+  static constexpr int kBytes = kMiscOffset + kMiscBytes + 1024;  // + alignment slack
+  static constexpr int kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+};
+
+__device__ __forceinline__ float load_weight(const void* w, int dt, int f) {
+  if (w == nullptr) return 1.0f;
+  if (dt == 4) return static_cast<const float*>(w)[f];
+  if (dt == 0) return __bfloat162float(static_cast<const __nv_bfloat16*>(w)[f]);
+  return __half2float(static_cast<const __half*>(w)[f]);
+}
+
+// Bounded wait that ignores the abort flag: used while unwinding, to let
+// copies and MMAs already in flight land before the CTA exits.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > kWaitTimeoutNs) {
+      set_device_error(kErrWaitTimeout);
+      return;
+    }
+  }
+}
+
+template <int BN, int STAGES, bool S1, bool FP8>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+  using L = GemmSmem<BN, STAGES>;
+  constexpr int KE = FP8 ? 128 : 64;  // K elements per stage
+  constexpr int kUmmaKBytes = 32;     // K bytes per MMA: 16 bf16 or 32 e4m3
+  constexpr uint32_t kIdesc = FP8 ? idesc_e4m3(kTileM, BN) : idesc_bf16(kTileM, BN);
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
+  static_assert(STAGES <= 32, "stage mask");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ok_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* rows_sm = reinterpret_cast<int*>(tmem_slot + 4);
+  int* last_sm = rows_sm + BN;
+  float* amax_part = reinterpret_cast<float*>(last_sm + BN);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], kEpiThreads);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  int n_blocks = g.sorted_ids ? (*g.num_padded) / BN : g.identity_rows / BN;
+  if (n_blocks > g.cap_blocks) n_blocks = g.cap_blocks;
+  const int total = n_blocks * g.n_mt;
+  const int slots = g.T * g.top_k;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_w = policy_evict_first();  // weights stream through once
+    const uint64_t pol_x = policy_evict_last();   // token rows are re-read per weight tile
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t pending = 0, pend_parity = 0;  // stages armed and not yet re-acquired
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int blk = tile / g.n_mt;
+      const int mt = tile - blk * g.n_mt;
+      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+      if (S1) {
+        for (int i = lane; i < BN; i += 32) {
+          const int r = blk * BN + i;
+          int row = 0;
+          if (!g.sorted_ids) {
+            row = r < g.T ? r : 0;
+          } else {
+            const int f = g.sorted_ids[r];
+            if (f >= 0 && f < slots) row = f / g.top_k;
+            else if (f != slots) set_device_error(kErrSlotRange);
+          }
+          rows_sm[i] = row;
+        }
+        __syncwarp();
+      }
+      for (int kb = 0; kb < g.num_kb; ++kb) {
+        if (lane == 0) {
+          ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
+          if (ok) {
+            pending &= ~(1u << stage);
+            uint8_t* a_dst = smem + stage * L::kStageBytes;
+            uint8_t* b_dst = a_dst + L::kABytes;
+            mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+            if (S1) {
+              tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+#pragma unroll 4
+              for (int q = 0; q < BN / 4; ++q)
+                tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
+                            rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
+            } else {
+              tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
+              tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+            }
+            pending |= 1u << stage;
+            pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if ((pending >> s) & 1u) drain_wait(&full[s], (pend_parity >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < g.num_kb; ++kb) {
+        if (lane == 0) ok = mbar_wait(&full[stage], phase, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + L::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < kTileKBytes / kUmmaKBytes; ++kk) {
+            // +32 bytes along K inside the swizzle row: +2 in the (addr >> 4) field
+            const uint64_t adv = static_cast<uint64_t>(kk * (kUmmaKBytes >> 4));
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (FP8)
+              umma_f8(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
+            else
+              umma_f16(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
+          }
+          umma_commit(&empty[stage]);  // smem stage free once these MMAs finish
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&acc_full[acc]);
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (!ok && lane == 0) {
+      umma_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;           // TMEM lane quarter this warp may read
+    const int et = threadIdx.x - 64;  // 0..127
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const int blk = tile / g.n_mt;
+      const int mt = tile - blk * g.n_mt;
+      if (et == 0) *ok_flag = mbar_wait(&acc_full[acc], acc_phase, abort_flag) ? 1 : 0;
+      named_bar_sync(kEpiBar, kEpiThreads);
+      const bool ok = *ok_flag != 0;
+      named_bar_sync(kEpiBar, kEpiThreads);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
+      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+
+      if (S1) {
+        // Lanes 0..15 of quarter q hold gate features 16q..16q+15 of this
+        // 64-feature tile, lanes 16..31 the matching up features.
+        const int feat = mt * 64 + 16 * q + (lane & 15);
+        const bool lo = lane < 16;
+        const float wsc = FP8 ? g.w_scale[expert] : 1.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
+          tmem_wait_ld();
+          if (c0 + 16 >= BN) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const float o0 = __shfl_xor_sync(0xffffffffu, v[i], 16);
+            const float o1 = __shfl_xor_sync(0xffffffffu, v[i + 1], 16);
+            float gt = lo ? v[i] : o1;
+            float up = lo ? o0 : v[i + 1];
+            const int c = c0 + i + (lo ? 0 : 1);
+            const int r = blk * BN + c;
+            if (FP8) {
+              int tok = r;
+              if (g.sorted_ids) {
+                const int f = g.sorted_ids[r];
+                tok = (f >= 0 && f < slots) ? f / g.top_k : 0;
+              } else if (tok >= g.T) {
+                tok = 0;
+              }
+              const float s = g.x_scale[tok] * wsc;
+              gt *= s;
+              up *= s;
+            }
+            const float hv = gt / (1.0f + expf(-gt)) * up;
+            if (feat < g.I) g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
+            if (FP8) {
+              // per-row amax of this tile's 16 features of the half-warp
+              float m = fabsf(hv);
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+              if ((lane & 15) == 0) amax_part[q * BN + c] = m;
+            }
+          }
+        }
+        if (FP8) {
+          named_bar_sync(kEpiBar, kEpiThreads);
+          for (int c = et; c < BN; c += kEpiThreads) {
+            const float m = fmaxf(fmaxf(amax_part[c], amax_part[BN + c]),
+                                  fmaxf(amax_part[2 * BN + c], amax_part[3 * BN + c]));
+            g.h_amax[static_cast<size_t>(mt) * g.rows_cap + blk * BN + c] = m;
+          }
+          named_bar_sync(kEpiBar, kEpiThreads);
+        }
+      } else {
+        const int n = mt * kTileM + 32 * q + lane;  // output feature
+        const bool nvalid = n < g.H;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
+          tmem_wait_ld();
+          if (c0 + 16 >= BN) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = blk * BN + c0 + i;
+            int f, t;
+            if (!g.sorted_ids) {
+              f = r;
+              t = r;
+              if (r >= g.T) continue;
+            } else {
+              f = g.sorted_ids[r];
+              if (f < 0 || f >= slots) continue;
+              t = f / g.top_k;
+            }
+            const float wt = load_weight(g.weights, g.weights_dtype, f);
+            const float val = v[i] * wt;
+            if (!nvalid) continue;
+            const size_t o = static_cast<size_t>(t) * g.H + n;
+            if (g.top_k == 1) {
+              float y = val;
+              if (g.addend) y += __bfloat162float(g.addend[o]);
+              g.out[o] = __float2bfloat16_rn(y);
+            } else {
+              red_add_f32(g.ws + o, val);
+            }
+          }
+        }
+        if (g.top_k > 1) {
+          // Arrival count per (token, weight tile): the epilogue that brings
+          // the k-th slot finalises the token's 128 outputs of this tile.
+          __threadfence();
+          named_bar_sync(kEpiBar, kEpiThreads);
+          for (int c = et; c < BN; c += kEpiThreads) {
+            const int f = g.sorted_ids[blk * BN + c];
+            int flag = 0;
+            if (f >= 0 && f < slots) {
+              int* cnt = g.counters + static_cast<size_t>(f / g.top_k) * g.n_mt + mt;
+              __threadfence();
+              if (atomicAdd(cnt, 1) == g.top_k - 1) {
+                flag = 1;
+                *cnt = 0;
+              }
+            }
+            last_sm[c] = flag;
+          }
+          named_bar_sync(kEpiBar, kEpiThreads);
+          __threadfence();
+          for (int c = 0; c < BN; ++c) {
+            if (!last_sm[c]) continue;
+            const int t = g.sorted_ids[blk * BN + c] / g.top_k;
+            if (nvalid) {
+              const size_t o = static_cast<size_t>(t) * g.H + n;
+              float y = atomicExch(g.ws + o, 0.0f);
+              if (g.addend) y += __bfloat162float(g.addend[o]);
+              g.out[o] = __float2bfloat16_rn(y);
+            }
+          }
+          named_bar_sync(kEpiBar, kEpiThreads);
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,395 @@
+// moe_b200.cu - C ABI of the routed + shared-expert MoE layer (include/moe_b200.h).
+//
+// Host side of every call: validate the arguments (nothing is launched on an
+// invalid argument), encode the TMA tensor maps, pick the kernel instance and
+// launch it on the caller's stream. All kernels live in the headers included
+// below and are compiled into this one translation unit.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include "moe_b200.h"
+#include "gate.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "router.cuh"
+#include "sort.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+moe_status_t fail_cuda(cudaError_t e, const char* what) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CK(call)                                     \
+  do {                                                   \
+    cudaError_t e_ = (call);                             \
+    if (e_ != cudaSuccess) return fail_cuda(e_, #call);  \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+inline bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128 || bm == 256; }
+
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    int v = cache[dev].load();
+    if (v) return v;
+  }
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cache[dev].store(n);
+  return n;
+}
+
+// ------------------------------------------------------------ TMA tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load();
+  if (f) return f;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult qr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) != cudaSuccess ||
+      qr != cudaDriverEntryPointSuccess || p == nullptr)
+    return nullptr;
+  f = reinterpret_cast<EncodeTiledFn>(p);
+  fn.store(f);
+  return f;
+}
+
+// Tiled map with the 128-byte swizzle; dims/box innermost first, strides in
+// bytes for dims 1..rank-1.
+moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+                      const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
+    return MOE_ERR_CUDA;
+  }
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = f(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (CUresult %d)",
+             static_cast<int>(r));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------ GEMM dispatch
+
+template <int BN>
+constexpr int stages_for() {
+  // ~192 KB of pipeline per CTA, one CTA per SM
+  return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : BN == 128 ? 6 : 4;
+}
+
+template <int BN, bool S1, bool FP8>
+moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
+                            cudaStream_t s) {
+  constexpr int ST = stages_for<BN>();
+  using L = moe::GemmSmem<BN, ST>;
+  auto kern = moe::k_moe_gemm<BN, ST, S1, FP8>;
+  static std::atomic<int> attr_set[64];
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load()) {
+    MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+  }
+  int grid = max_tiles < num_sms() ? max_tiles : num_sms();
+  if (grid < 1) grid = 1;
+  kern<<<grid, moe::kGemmThreads, L::kBytes, s>>>(ta, tb, g);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+template <bool S1, bool FP8>
+moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g,
+                         int max_tiles, cudaStream_t s) {
+  switch (bm) {
+    case 16: return launch_gemm_bn<16, S1, FP8>(ta, tb, g, max_tiles, s);
+    case 32: return launch_gemm_bn<32, S1, FP8>(ta, tb, g, max_tiles, s);
+    case 64: return launch_gemm_bn<64, S1, FP8>(ta, tb, g, max_tiles, s);
+    case 128: return launch_gemm_bn<128, S1, FP8>(ta, tb, g, max_tiles, s);
+    case 256: return launch_gemm_bn<256, S1, FP8>(ta, tb, g, max_tiles, s);
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+// Padded sorted length bound T*k + E*(bm-1), rounded up to whole blocks.
+size_t capacity(int T, int k, int E, int bm) {
+  const size_t n = static_cast<size_t>(T) * k + static_cast<size_t>(E) * (bm - 1);
+  return (n + bm - 1) / bm * bm;
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_DTYPE: return "MOE_ERR_UNSUPPORTED_DTYPE";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_SHAPE: return "MOE_ERR_SHAPE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_supports_output_addend(void) { return 1; }
+
+moe_status_t moe_device_error(int* code, moe_stream_t stream) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  MOE_CK(cudaStreamSynchronize(as_stream(stream)));
+  int v = 0;
+  MOE_CK(cudaMemcpyFromSymbol(&v, moe::g_device_error, sizeof(int)));
+  const int zero = 0;
+  MOE_CK(cudaMemcpyToSymbol(moe::g_device_error, &zero, sizeof(int)));
+  *code = v;
+  return MOE_OK;
+}
+
+size_t moe_sorted_capacity(int T, int top_k, int E, int block_m) {
+  if (T < 0 || top_k < 0 || E < 0 || block_m < 1) return 0;
+  return capacity(T, top_k, E, block_m);
+}
+
+size_t moe_stage2_workspace_bytes(int T, int H) {
+  if (T < 1 || H < 1) return 0;
+  const size_t n_mt = (static_cast<size_t>(H) + moe::kTileM - 1) / moe::kTileM;
+  return static_cast<size_t>(T) * H * sizeof(float) + static_cast<size_t>(T) * n_mt * sizeof(int);
+}
+
+size_t moe_stage1_amax_bytes(int dtype, int rows, int I) {
+  if (dtype != MOE_DT_FP8_E4M3 || rows < 1 || I < 1) return 0;
+  return static_cast<size_t>((I + 63) / 64) * rows * sizeof(float);
+}
+
+moe_status_t moe_router_topk(const float* logits, const float* correction_bias, int T, int E, int top_k, int mode,
+                             int n_group, int topk_group, int renormalize, float routed_scaling_factor,
+                             int32_t* topk_ids, float* topk_weights, moe_stream_t stream) {
+  if (!logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOPK)
+    return MOE_ERR_INVALID_ARG;
+  if (mode != MOE_ROUTE_SOFTMAX && mode != MOE_ROUTE_GROUPED_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (mode == MOE_ROUTE_GROUPED_SIGMOID) {
+    if (n_group < 1 || n_group > 32 || E % n_group != 0) return MOE_ERR_INVALID_ARG;
+    if (topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+    if (top_k > topk_group * (E / n_group)) return MOE_ERR_INVALID_ARG;
+  } else if (correction_bias) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  moe::RouterArgs a{logits, correction_bias, T, E, top_k, mode, n_group, topk_group, renormalize,
+                    routed_scaling_factor, topk_ids, topk_weights};
+  const int vpl = (E + 31) / 32;
+  const dim3 grid((T + moe::kRouterWarps - 1) / moe::kRouterWarps);
+  const dim3 block(moe::kRouterWarps * 32);
+  const size_t smem = static_cast<size_t>(moe::kRouterWarps) * 2 * E * sizeof(float);
+  cudaStream_t s = as_stream(stream);
+  if (vpl <= 1) moe::k_router_topk<1><<<grid, block, smem, s>>>(a);
+  else if (vpl <= 2) moe::k_router_topk<2><<<grid, block, smem, s>>>(a);
+  else if (vpl <= 4) moe::k_router_topk<4><<<grid, block, smem, s>>>(a);
+  else if (vpl <= 8) moe::k_router_topk<8><<<grid, block, smem, s>>>(a);
+  else moe::k_router_topk<16><<<grid, block, smem, s>>>(a);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, int block_m, int32_t* sorted_ids,
+                            int32_t* block_expert, int32_t* expert_counts, int32_t* expert_offsets,
+                            int32_t* num_padded, moe_stream_t stream) {
+  if (!topk_ids || !sorted_ids || !block_expert || !expert_counts || !expert_offsets || !num_padded)
+    return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || E > MOE_MAX_EXPERTS || !valid_block_m(block_m)) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * top_k > (1ll << 20)) return MOE_ERR_SHAPE;
+  moe::SortArgs a{topk_ids, T * top_k, E, block_m, sorted_ids, block_expert, expert_counts, expert_offsets,
+                  num_padded};
+  const size_t smem = (2 * static_cast<size_t>(E) + 32 * static_cast<size_t>(E) + 32) * sizeof(int);
+  static std::atomic<int> attr_set[64];
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load()) {
+    MOE_CK(cudaFuncSetAttribute(moe::k_align_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>((2 + 32) * MOE_MAX_EXPERTS * sizeof(int) + 32 * sizeof(int))));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+  }
+  moe::k_align_sort<<<1, moe::kSortThreads, smem, as_stream(stream)>>>(a);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t shared_expert_gate_dot(int dtype, const void* x, const void* w, int T, int K, int apply_sigmoid,
+                                    void* out, moe_stream_t stream) {
+  if (!x || !w || !out || T < 1 || K < 1) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const int vec_ok = (K % 8 == 0) && aligned16(x) && aligned16(w);
+  cudaStream_t s = as_stream(stream);
+  if (dtype == MOE_DT_BF16)
+    moe::k_gate_dot<__nv_bfloat16><<<T, moe::kGateThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w), K, apply_sigmoid, vec_ok,
+        static_cast<__nv_bfloat16*>(out));
+  else
+    moe::k_gate_dot<__half><<<T, moe::kGateThreads, 0, s>>>(static_cast<const __half*>(x),
+                                                            static_cast<const __half*>(w), K, apply_sigmoid,
+                                                            vec_ok, static_cast<__half*>(out));
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, const void* w13,
+                             const float* w13_scale, const int32_t* sorted_ids, const int32_t* block_expert,
+                             const int32_t* num_padded, int T, int top_k, int H, int I, int E, int block_m, void* h,
+                             float* h_amax, moe_stream_t stream) {
+  const bool fp8 = dtype == MOE_DT_FP8_E4M3;
+  if (dtype != MOE_DT_BF16 && !fp8) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!x || !w13 || !h) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
+    return MOE_ERR_INVALID_ARG;
+  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
+  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!x_scale || !w13_scale || !h_amax)) return MOE_ERR_INVALID_ARG;
+  if (H % (fp8 ? 128 : 64) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(h)) return MOE_ERR_ALIGNMENT;
+
+  const int es = fp8 ? 1 : 2;
+  const int ke = fp8 ? 128 : 64;
+  const size_t rows_cap = sorted_ids ? capacity(T, top_k, E, block_m)
+                                     : static_cast<size_t>((T + block_m - 1) / block_m) * block_m;
+  const int cap_blocks = static_cast<int>((rows_cap + block_m - 1) / block_m);
+  const CUtensorMapDataType tdt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+  // W13 as 5-D (K, row-in-16, gate|up, 16-row group, expert): one box brings
+  // 16 gate rows then the 16 matching up rows for four consecutive groups, so
+  // the 128 weight rows of a tile pair gate and up inside each 32-lane quarter.
+  CUtensorMap ta, tb;
+  {
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(H), 16, 2, static_cast<cuuint64_t>(I / 16),
+                                static_cast<cuuint64_t>(E)};
+    const cuuint64_t st[4] = {static_cast<cuuint64_t>(H) * es, static_cast<cuuint64_t>(I) * H * es,
+                              16ull * H * es, 2ull * I * H * es};
+    const cuuint32_t box[5] = {static_cast<cuuint32_t>(ke), 16, 2, 4, 1};
+    moe_status_t r = make_map(&ta, tdt, 5, w13, dims, st, box);
+    if (r != MOE_OK) return r;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), 1};
+    moe_status_t r = make_map(&tb, tdt, 2, x, dims, st, box);
+    if (r != MOE_OK) return r;
+  }
+  moe::GemmArgs g{};
+  g.sorted_ids = sorted_ids;
+  g.block_expert = block_expert;
+  g.num_padded = num_padded;
+  g.identity_rows = static_cast<int>(rows_cap);
+  g.cap_blocks = cap_blocks;
+  g.T = T;
+  g.top_k = top_k;
+  g.H = H;
+  g.I = I;
+  g.n_mt = I / 64;
+  g.num_kb = H / ke;
+  g.h = static_cast<__nv_bfloat16*>(h);
+  g.h_amax = h_amax;
+  g.rows_cap = static_cast<int>(rows_cap);
+  g.x_scale = x_scale;
+  g.w_scale = w13_scale;
+  const int max_tiles = cap_blocks * g.n_mt;
+  cudaStream_t s = as_stream(stream);
+  return fp8 ? launch_gemm<true, true>(block_m, ta, tb, g, max_tiles, s)
+             : launch_gemm<true, false>(block_m, ta, tb, g, max_tiles, s);
+}
+
+moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h_amax, const void* w2,
+                                        const float* w2_scale, const void* weights, int weights_dtype,
+                                        const int32_t* sorted_ids, const int32_t* block_expert,
+                                        const int32_t* num_padded, int T, int top_k, int H, int I, int E,
+                                        int block_m, const void* addend, moe_event_t addend_ready, void* acc_ws,
+                                        void* out, moe_stream_t stream) {
+  if (dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  (void)h_amax;
+  (void)w2_scale;
+  if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
+    return MOE_ERR_INVALID_ARG;
+  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
+  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
+  if (top_k > 1 && !acc_ws) return MOE_ERR_INVALID_ARG;
+  if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
+    return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)) ||
+      (acc_ws && !aligned16(acc_ws)))
+    return MOE_ERR_ALIGNMENT;
+
+  const int es = 2;
+  const int ke = 64;
+  const size_t rows_cap = sorted_ids ? capacity(T, top_k, E, block_m)
+                                     : static_cast<size_t>((T + block_m - 1) / block_m) * block_m;
+  const int cap_blocks = static_cast<int>((rows_cap + block_m - 1) / block_m);
+  CUtensorMap ta, tb;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(E)};
+    const cuuint64_t st[2] = {static_cast<cuuint64_t>(I) * es, static_cast<cuuint64_t>(H) * I * es};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(moe::kTileM), 1};
+    moe_status_t r = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w2, dims, st, box);
+    if (r != MOE_OK) return r;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(cap_blocks) * block_m};
+    const cuuint64_t st[1] = {static_cast<cuuint64_t>(I) * es};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
+    moe_status_t r = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, dims, st, box);
+    if (r != MOE_OK) return r;
+  }
+  cudaStream_t s = as_stream(stream);
+  if (addend_ready) MOE_CK(cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(addend_ready), 0));
+
+  moe::GemmArgs g{};
+  g.sorted_ids = sorted_ids;
+  g.block_expert = block_expert;
+  g.num_padded = num_padded;
+  g.identity_rows = static_cast<int>(rows_cap);
+  g.cap_blocks = cap_blocks;
+  g.T = T;
+  g.top_k = top_k;
+  g.H = H;
+  g.I = I;
+  g.n_mt = H / moe::kTileM;
+  g.num_kb = I / ke;
+  g.weights = weights;
+  g.weights_dtype = weights_dtype;
+  g.addend = static_cast<const __nv_bfloat16*>(addend);
+  g.ws = static_cast<float*>(acc_ws);
+  g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
+  g.out = static_cast<__nv_bfloat16*>(out);
+  const int max_tiles = cap_blocks * g.n_mt;
+  return launch_gemm<false, false>(block_m, ta, tb, g, max_tiles, s);
+}
+
+}  // extern "C"

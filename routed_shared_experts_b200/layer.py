@@ -1,0 +1,106 @@
+"""One MoE layer forward composed from the five C-ABI calls.
+
+Main stream: router top-k -> align/sort -> stage 1 -> stage 2 (waits on the
+addend event right before its GEMM). Side stream: shared gate -> shared stage 1
+-> shared stage 2 (identity routing, top_k = 1, row weight = gate) writing the
+bf16 addend -> record the addend event. This is the schedule of vllm-project/
+vllm PR 65207 "Purpose", commit 2: the aux-stream shared expert overlaps
+sorting and stage 1, and stage 2 accumulates its output in the epilogue.
+
+PyTorch provides the device buffers, streams and events only; every step runs
+in ``libmoe_b200.so``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import capi
+from .configs import MoEConfig
+
+
+class MoELayer:
+    """Device buffers and weights of one layer; ``forward()`` enqueues a step.
+
+    ``inp`` is a dict from ``synth.make_layer_inputs`` (tensors already on the
+    device). Weights are referenced, not copied; activations (``x``,
+    ``logits``) are read from the same dict at every forward, so a caller may
+    refill them in place.
+    """
+
+    def __init__(self, cfg: MoEConfig, inp: dict, block_m: int | None = None, device=None):
+        self.cfg = cfg
+        self.inp = inp
+        self.device = torch.device(device or inp["x"].device)
+        dev = self.device
+        T, H, E, k, I, Is = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I, cfg.Is
+        self.bm = block_m or cfg.block_m
+        self.dt = capi.DTYPES[cfg.dtype]
+        bm = self.bm
+        cap = capi.sorted_capacity(T, k, E, bm)
+        cap_s = capi.sorted_capacity(T, 1, 1, bm)  # identity rows of the shared expert
+        self.cap = cap
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.topk_ids = torch.empty((T, k), **i32)
+        self.topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.sorted_ids = torch.empty(cap, **i32)
+        self.block_expert = torch.empty(cap // bm, **i32)
+        self.expert_counts = torch.empty(E, **i32)
+        self.expert_offsets = torch.empty(E + 1, **i32)
+        self.num_padded = torch.empty(1, **i32)
+        self.h = torch.empty((cap, I), dtype=torch.bfloat16, device=dev)
+        self.h_s = torch.empty((cap_s, Is), dtype=torch.bfloat16, device=dev)
+        amax_b = capi.stage1_amax_bytes(self.dt, cap, I)
+        amax_bs = capi.stage1_amax_bytes(self.dt, cap_s, Is)
+        self.h_amax = torch.empty(max(amax_b // 4, 1), dtype=torch.float32, device=dev) if amax_b else None
+        self.h_amax_s = torch.empty(max(amax_bs // 4, 1), dtype=torch.float32, device=dev) if amax_bs else None
+        gdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float16
+        self.gate = torch.empty(T, dtype=gdt, device=dev) if cfg.shared_gate else None
+        self.addend = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ws = capi.stage2_workspace_bytes(T, H)
+        self.acc_ws = torch.zeros(ws // 4, dtype=torch.float32, device=dev)  # zeroed once
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_in = torch.cuda.Event()
+        self.ev_addend = torch.cuda.Event()
+
+    # -- the two halves -------------------------------------------------------
+
+    def shared_expert(self, stream):
+        cfg, inp = self.cfg, self.inp
+        T, H, Is = cfg.T, cfg.H, cfg.Is
+        if self.gate is not None:
+            capi.shared_expert_gate_dot(capi.MOE_DT_BF16, inp["x"], inp["w_gate"], True, self.gate, stream)
+        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13s"], inp.get("w13s_scale"),
+                             None, None, None, T, 1, H, Is, 1, self.bm, self.h_s, self.h_amax_s, stream)
+        wdt = capi.MOE_DT_BF16 if self.gate is not None else capi.MOE_DT_F32
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_amax_s, inp["w2s"], inp.get("w2s_scale"),
+                                        self.gate, wdt, None, None, None, T, 1, H, Is, 1, self.bm, None, None,
+                                        None, self.addend, stream)
+
+    def routed(self, stream, addend=True):
+        cfg, inp = self.cfg, self.inp
+        T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I
+        mode = capi.MOE_ROUTE_SOFTMAX if cfg.route == "softmax" else capi.MOE_ROUTE_GROUPED_SIGMOID
+        capi.moe_router_topk(inp["logits"], inp.get("correction_bias"), k, mode, cfg.n_group, cfg.topk_group,
+                             cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, stream)
+        capi.moe_align_sort(self.topk_ids, E, self.bm, self.sorted_ids, self.block_expert, self.expert_counts,
+                            self.expert_offsets, self.num_padded, stream)
+        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], inp.get("w13_scale"),
+                             self.sorted_ids, self.block_expert, self.num_padded, T, k, H, I, E, self.bm, self.h,
+                             self.h_amax, stream)
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_amax, inp["w2"], inp.get("w2_scale"),
+                                        self.topk_weights, capi.MOE_DT_F32, self.sorted_ids, self.block_expert,
+                                        self.num_padded, T, k, H, I, E, self.bm,
+                                        self.addend if addend else None, self.ev_addend if addend else None,
+                                        self.acc_ws, self.out, stream)
+
+    def forward(self, stream=None):
+        """Enqueue one layer step on ``stream`` (default: current stream);
+        returns ``self.out``. Capturable in a CUDA graph."""
+        main = stream or torch.cuda.current_stream(self.device)
+        self.ev_in.record(main)
+        self.side.wait_event(self.ev_in)
+        self.shared_expert(self.side)
+        self.ev_addend.record(self.side)
+        self.routed(main)
+        return self.out

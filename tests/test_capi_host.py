@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function ``include/moe_b200.h`` declares, and rejects invalid arguments
+with the documented status before touching the device.
+
+Invalid-argument calls pass fake device addresses; they must be refused on the
+host, so these tests run only where no GPU is present (a missing check would
+otherwise reach a launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from routed_shared_experts_b200 import build, capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return capi.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+|shared_expert_gate_dot)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "moe_stage2_gemm_accumulate" in names and "shared_expert_gate_dot" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(capi.SIGNATURES)
+
+
+def test_info_calls(lib):
+    assert lib.moe_supports_output_addend() == 1
+    assert b"sm_100a" in lib.moe_version()
+    assert lib.moe_status_string(-1) == b"MOE_ERR_INVALID_ARG"
+    assert lib.moe_sorted_capacity(32, 8, 128, 16) == 32 * 8 + 128 * 15  # already a multiple of 16
+    assert lib.moe_sorted_capacity(5, 3, 7, 64) == 512  # 15 + 441 = 456 -> 512
+    assert lib.moe_stage2_workspace_bytes(32, 2048) == 32 * 2048 * 4 + 32 * 16 * 4
+    assert lib.moe_stage1_amax_bytes(capi.MOE_DT_FP8_E4M3, 100, 1408) == 22 * 100 * 4
+    assert lib.moe_stage1_amax_bytes(capi.MOE_DT_BF16, 100, 1408) == 0
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake device addresses: CPU-only check")
+P = 0x10000  # 16-byte aligned fake address, never dereferenced on the host
+
+
+@no_gpu
+def test_router_rejects(lib):
+    f = lib.moe_router_topk
+    ok = dict(l=P, b=None, T=4, E=8, k=2, mode=0, ng=1, tg=1, rn=1, rsf=1.0, ids=P, w=P)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["l"], a["b"], a["T"], a["E"], a["k"], a["mode"], a["ng"], a["tg"], a["rn"], a["rsf"], a["ids"],
+                 a["w"], None)
+    assert call(l=None) == -1
+    assert call(T=0) == -1
+    assert call(E=513) == -1
+    assert call(k=9) == -1
+    assert call(k=33, E=64) == -1
+    assert call(mode=2) == -1
+    assert call(b=P) == -1                          # bias only in grouped mode
+    assert call(mode=1, ng=3) == -1                 # 3 does not divide 8
+    assert call(mode=1, ng=4, tg=5) == -1
+    assert call(mode=1, ng=4, tg=1, k=3) == -1      # k > topk_group * E / n_group
+
+
+@no_gpu
+def test_sort_rejects(lib):
+    f = lib.moe_align_sort
+    assert f(None, 4, 2, 8, 16, P, P, P, P, P, None) == -1
+    assert f(P, 4, 2, 8, 48, P, P, P, P, P, None) == -1       # block_m not in the set
+    assert f(P, 4, 2, 600, 16, P, P, P, P, P, None) == -1     # E too large
+    assert f(P, 1 << 19, 4, 8, 16, P, P, P, P, P, None) == -4  # too many slots
+
+
+@no_gpu
+def test_gate_rejects(lib):
+    f = lib.shared_expert_gate_dot
+    assert f(capi.MOE_DT_F32, P, P, 1, 8, 1, P, None) == -2
+    assert f(capi.MOE_DT_BF16, None, P, 1, 8, 1, P, None) == -1
+    assert f(capi.MOE_DT_BF16, P, P, 0, 8, 1, P, None) == -1
+
+
+@no_gpu
+def test_stage1_rejects(lib):
+    f = lib.moe_stage1_gemm
+
+    def call(dt=0, x=P, xs=None, w=P, ws=None, s=P, be=P, npd=P, T=4, k=2, H=256, I=128, E=8, bm=16, h=P, am=None):
+        return f(dt, x, xs, w, ws, s, be, npd, T, k, H, I, E, bm, h, am, None)
+    assert call(dt=capi.MOE_DT_F32) == -2
+    assert call(x=None) == -1
+    assert call(bm=24) == -1
+    assert call(be=None) == -1
+    assert call(s=None) == -1                       # identity routing needs top_k == 1
+    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales and the amax buffer
+    assert call(H=200) == -4
+    assert call(I=100) == -4
+    assert call(x=P + 8) == -3
+
+
+@no_gpu
+def test_stage2_rejects(lib):
+    f = lib.moe_stage2_gemm_accumulate
+
+    def call(dt=0, h=P, am=None, w2=P, w2s=None, wt=P, wdt=capi.MOE_DT_F32, s=P, be=P, npd=P, T=4, k=2, H=256,
+             I=128, E=8, bm=16, add=None, ev=None, ws=P, out=P):
+        return f(dt, h, am, w2, w2s, wt, wdt, s, be, npd, T, k, H, I, E, bm, add, ev, ws, out, None)
+    assert call(dt=capi.MOE_DT_FP16) == -2
+    assert call(out=None) == -1
+    assert call(ws=None) == -1                      # top_k > 1 needs the workspace
+    assert call(wdt=7) == -2
+    assert call(H=200) == -4
+    assert call(out=P + 4) == -3
+    assert call(add=P + 2) == -3
+    assert call(s=None) == -1
