@@ -77,7 +77,9 @@ class MoELayer:
                                         self.gate, wdt, None, None, None, T, 1, H, Is, 1, self.bm, None, None,
                                         None, self.addend, stream)
 
-    def routed(self, stream, addend=True):
+    def routed(self, stream, addend=True, probes=None):
+        """Main-stream half. ``probes`` = optional four events recorded on
+        ``stream`` right before/after stage 1 and right before/after stage 2."""
         cfg, inp = self.cfg, self.inp
         T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I
         mode = capi.MOE_ROUTE_SOFTMAX if cfg.route == "softmax" else capi.MOE_ROUTE_GROUPED_SIGMOID
@@ -85,16 +87,25 @@ class MoELayer:
                              cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, stream)
         capi.moe_align_sort(self.topk_ids, E, self.bm, self.sorted_ids, self.block_expert, self.expert_counts,
                             self.expert_offsets, self.num_padded, stream)
+        if probes:
+            probes[0].record(stream)
         capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], inp.get("w13_scale"),
                              self.sorted_ids, self.block_expert, self.num_padded, T, k, H, I, E, self.bm, self.h,
                              self.h_amax, stream)
+        if probes:
+            probes[1].record(stream)
+            if addend:  # take the addend wait before the probe: the pair times the kernel alone
+                stream.wait_event(self.ev_addend)
+            probes[2].record(stream)
         capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_amax, inp["w2"], inp.get("w2_scale"),
                                         self.topk_weights, capi.MOE_DT_F32, self.sorted_ids, self.block_expert,
                                         self.num_padded, T, k, H, I, E, self.bm,
                                         self.addend if addend else None, self.ev_addend if addend else None,
                                         self.acc_ws, self.out, stream)
+        if probes:
+            probes[3].record(stream)
 
-    def forward(self, stream=None):
+    def forward(self, stream=None, probes=None):
         """Enqueue one layer step on ``stream`` (default: current stream);
         returns ``self.out``. Capturable in a CUDA graph."""
         main = stream or torch.cuda.current_stream(self.device)
@@ -102,5 +113,10 @@ class MoELayer:
         self.side.wait_event(self.ev_in)
         self.shared_expert(self.side)
         self.ev_addend.record(self.side)
-        self.routed(main)
+        self.routed(main, probes=probes)
         return self.out
+
+    # kernels this library launches per forward()
+    @property
+    def launches_per_step(self) -> int:
+        return 6 + (1 if self.gate is not None else 0)

@@ -50,7 +50,7 @@ def test_router_grouped_config(cuda_lib, name):
 
 
 @pytest.mark.parametrize("E,k,n_group,topk_group", [(256, 8, 8, 4), (8, 2, 1, 1), (16, 16, 4, 4), (512, 32, 32, 8),
-                                                    (64, 1, 64, 1)])
+                                                    (64, 1, 32, 1)])
 def test_router_grouped_shapes_with_ties(cuda_lib, E, k, n_group, topk_group):
     g = torch.Generator().manual_seed(E + k)
     # quantised logits create exact ties in c and in the group scores

@@ -35,9 +35,10 @@ def _check_layer(cfg, block_m=None, tokens=None):
         g = layer.gate.float().cpu().numpy()[tok]
         assert np.all(np.abs(g - ref["gate"]) <= 2.0**-8 * np.abs(ref["gate"]) + 1e-12)
     add = layer.addend.float().cpu().numpy()[tok]
-    assert_close_rms(add, ref["addend"], BF16_TOL, "addend")
+    assert_close_rms(add, ref["addend"], BF16_TOL, "addend", exact_frac=0.9)
     out = layer.out.float().cpu().numpy()[tok]
-    rel = assert_close_rms(out, ref["out"], BF16_TOL, "out")
+    rel = assert_close_rms(out, ref["out"], BF16_TOL, "out", rounded=[ref["out"], ref["addend"]],
+                           exact_frac=0.9)
     # the stage-2 workspace is left zeroed for the next call
     assert torch.count_nonzero(layer.acc_ws).item() == 0
     return layer, ref, rel
@@ -96,8 +97,12 @@ def test_addend_in_epilogue_equals_separate_add(cuda_lib):
     main = torch.cuda.current_stream()
     layer.routed(main, addend=False)
     torch.cuda.synchronize()
-    separate = layer.out.float() + layer.addend.float()
-    assert_close_rms(fused.cpu().numpy(), separate.cpu().numpy(), BF16_TOL, "fused vs separate")
+    routed = layer.out.float().cpu().numpy()
+    addend = layer.addend.float().cpu().numpy()
+    # fused rounds (addend + routed sum) once; the separate path rounded the
+    # routed sum first: one bf16 step of each may separate them
+    assert_close_rms(fused.cpu().numpy(), routed + addend, BF16_TOL, "fused vs separate",
+                     rounded=[routed + addend, routed])
 
 
 def test_rsf_fold_scales_routed_output(cuda_lib):
@@ -110,7 +115,7 @@ def test_rsf_fold_scales_routed_output(cuda_lib):
         layer.routed(torch.cuda.current_stream(), addend=False)
         torch.cuda.synchronize()
         outs.append(layer.out.float().cpu().numpy())
-    assert_close_rms(outs[1], 2.5 * outs[0], BF16_TOL, "rsf fold")
+    assert_close_rms(outs[1], 2.5 * outs[0], BF16_TOL, "rsf fold", rounded=[outs[1], 2.5 * outs[0]])
 
 
 def test_cuda_graph_replay(cuda_lib):
@@ -130,7 +135,8 @@ def test_cuda_graph_replay(cuda_lib):
         graph.replay()
     torch.cuda.synchronize()
     assert capi.device_error() == 0
-    assert_close_rms(layer.out.float().cpu().numpy(), eager.cpu().numpy(), 2.0**-7, "graph vs eager")
+    assert_close_rms(layer.out.float().cpu().numpy(), eager.cpu().numpy(), BF16_TOL, "graph vs eager",
+                     exact_frac=0.95)
     assert torch.count_nonzero(layer.acc_ws).item() == 0
     del graph
 
@@ -140,4 +146,5 @@ def test_repeated_steps_are_stable(cuda_lib):
     inp = synth.make_layer_inputs(cfg)
     layer = run_layer(cfg, to_dev(inp), steps=5)
     ref = oracle_layer(cfg, inp, tokens=np.arange(0, cfg.T, 4))
-    assert_close_rms(layer.out.float().cpu().numpy()[ref["tokens"]], ref["out"], BF16_TOL, "after 5 steps")
+    assert_close_rms(layer.out.float().cpu().numpy()[ref["tokens"]], ref["out"], BF16_TOL, "after 5 steps",
+                     rounded=[ref["out"], ref["addend"]], exact_frac=0.9)
