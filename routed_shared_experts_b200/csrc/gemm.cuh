@@ -8,8 +8,9 @@
 //               rows are gathered from x by TMA gather4 through sorted_ids.
 //   warp 1      TMEM allocator + MMA issuer (one thread): tcgen05.mma with the
 //               weights as A (M = 128) and the tokens as B (N = BN), fp32
-//               accumulator in TMEM, double-buffered across tiles.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, then
+//               accumulator in TMEM, a ring of 2 or 4 across tiles.
+//   warps 2..  epilogue, one or two warpgroups taking alternate tiles:
+//               tcgen05.ld of the accumulator, then
 //               stage 1: optional fp8 scales, SiLU(gate) * up, store h;
 //               stage 2: scales x top-k weight, fp32 red.add into the token
 //               row, and the CTA that brings a token's last slot adds the
@@ -29,11 +30,19 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 192;
 constexpr int kTileM = 128;       // weight rows per tile = MMA M
 constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte swizzle row
-constexpr int kEpiThreads = 128;
-constexpr int kEpiBar = 1;        // named barrier of the 4 epilogue warps
+constexpr int kEpiThreads = 128;  // one epilogue warpgroup
+
+// Epilogue warpgroups per CTA: two groups take alternate tiles (each with two
+// TMEM accumulators) so a tile's epilogue - atomics to L2 included - overlaps
+// the next tiles' main loop; 256-token tiles fill TMEM with two accumulators.
+template <int BN>
+struct EpiCfg {
+  static constexpr int kGroups = BN <= 128 ? 2 : 1;
+  static constexpr int kAcc = 2 * kGroups;
+  static constexpr int kThreads = 64 + kEpiThreads * kGroups;
+};
 
 struct GemmArgs {
   const int32_t* sorted_ids;  // nullptr: identity routing (row r = token r, expert 0)
@@ -63,17 +72,21 @@ struct GemmArgs {
 
 template <int BN, int STAGES>
 struct GemmSmem {
+  static constexpr int kGroups = EpiCfg<BN>::kGroups;
+  static constexpr int kAcc = EpiCfg<BN>::kAcc;
   static constexpr int kABytes = kTileM * kTileKBytes;
   static constexpr int kBBytes = BN * kTileKBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  // full[S], empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr int kNumBars = 2 * STAGES + 5;
+  // full[S], empty[S], acc_full[A], acc_empty[A], drain
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
-  // tmem slot, abort flag, ok flag, pad, rows[BN], last[BN], amax_part[4][BN]
-  static constexpr int kMiscBytes = 16 + BN * 4 + BN * 4 + 4 * BN * 4;
+  // tmem slot, abort flag, 2 pad words, producer rows[BN]; then per epilogue
+  // group: ok flag + 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
+  static constexpr int kGroupWords = 4 + 7 * BN;
+  static constexpr int kMiscBytes = 16 + BN * 4 + kGroups * kGroupWords * 4;
   static constexpr int kBytes = kMiscOffset + kMiscBytes + 1024;  // + alignment slack
-  static constexpr int kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+  static constexpr int kTmemCols = (kAcc * BN < 32) ? 32 : kAcc * BN;
 };
 
 __device__ __forceinline__ float load_weight(const void* w, int dt, int f) {
@@ -96,10 +109,18 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 template <int BN, int STAGES, bool S1, bool FP8>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
     k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
   using L = GemmSmem<BN, STAGES>;
+  constexpr int G = L::kGroups;
+  constexpr int NACC = L::kAcc;
   constexpr int KE = FP8 ? 128 : 64;  // K elements per stage
   constexpr int kUmmaKBytes = 32;     // K bytes per MMA: 16 bf16 or 32 e4m3
   constexpr uint32_t kIdesc = FP8 ? idesc_e4m3(kTileM, BN) : idesc_bf16(kTileM, BN);
@@ -111,14 +132,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + NACC;
+  uint64_t* drain = acc_empty + NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* ok_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* rows_sm = reinterpret_cast<int*>(tmem_slot + 4);
-  int* last_sm = rows_sm + BN;
-  float* amax_part = reinterpret_cast<float*>(last_sm + BN);
+  int* group_base = rows_sm + BN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -128,7 +147,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NACC; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], kEpiThreads);
     }
@@ -216,10 +235,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    int j = 0;  // local tile counter: accumulator j % NACC, use (j / NACC)
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+      const int acc = j % NACC;
+      const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
       if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -255,10 +275,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) break;
       if (lane == 0) umma_commit(&acc_full[acc]);
       __syncwarp();
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
     }
     if (!ok && lane == 0) {
       umma_commit(drain);
@@ -266,28 +282,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;           // TMEM lane quarter this warp may read
-    const int et = threadIdx.x - 64;  // 0..127
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const int grp = (warp - 2) >> 2;              // epilogue group: tiles j with j % G == grp
+    const int q = warp & 3;                       // TMEM lane quarter this warp may read
+    const int et = threadIdx.x - 64 - kEpiThreads * grp;  // 0..127 inside the group
+    const int bar_id = 1 + grp;                   // named barrier of this group
+    int* gsm = group_base + grp * L::kGroupWords;
+    volatile int* ok_sm = gsm;
+    int* tok_sm = gsm + 4;                        // token of each column, -1 = padding
+    float* wgt_sm = reinterpret_cast<float*>(tok_sm + BN);  // stage 2: top-k weight; stage 1 fp8: x scale
+    int* last_sm = reinterpret_cast<int*>(wgt_sm + BN);
+    float* amax_part = reinterpret_cast<float*>(last_sm + BN);
+    int j = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+      if (j % G != grp) continue;
       const int blk = tile / g.n_mt;
       const int mt = tile - blk * g.n_mt;
-      if (et == 0) *ok_flag = mbar_wait(&acc_full[acc], acc_phase, abort_flag) ? 1 : 0;
-      named_bar_sync(kEpiBar, kEpiThreads);
-      const bool ok = *ok_flag != 0;
-      named_bar_sync(kEpiBar, kEpiThreads);
-      if (!ok) break;
+      const int acc = j % NACC;
+      const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
+      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+
+      // per-column metadata, fetched while the accumulator is still being built
+      for (int c = et; c < BN; c += kEpiThreads) {
+        const int r = blk * BN + c;
+        int f = r, t = -1;
+        if (!g.sorted_ids) {
+          if (r < g.T) t = r;
+        } else {
+          f = g.sorted_ids[r];
+          if (f >= 0 && f < slots) t = f / g.top_k;
+        }
+        tok_sm[c] = t;
+        float w = 0.f;
+        if (t >= 0) {
+          if (S1) w = FP8 ? g.x_scale[t] * g.w_scale[expert] : 1.0f;
+          else w = load_weight(g.weights, g.weights_dtype, f);
+        }
+        wgt_sm[c] = w;
+      }
+      if (et == 0) *ok_sm = mbar_wait(&acc_full[acc], acc_phase, abort_flag) ? 1 : 0;
+      named_bar_sync(bar_id, kEpiThreads);
+      if (!*ok_sm) break;  // same value in every thread of the group
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN);
-      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
 
       if (S1) {
         // Lanes 0..15 of quarter q hold gate features 16q..16q+15 of this
         // 64-feature tile, lanes 16..31 the matching up features.
         const int feat = mt * 64 + 16 * q + (lane & 15);
         const bool lo = lane < 16;
-        const float wsc = FP8 ? g.w_scale[expert] : 1.0f;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
@@ -306,16 +348,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int c = c0 + i + (lo ? 0 : 1);
             const int r = blk * BN + c;
             if (FP8) {
-              int tok = r;
-              if (g.sorted_ids) {
-                const int f = g.sorted_ids[r];
-                tok = (f >= 0 && f < slots) ? f / g.top_k : 0;
-              } else if (tok >= g.T) {
-                tok = 0;
-              }
-              const float s = g.x_scale[tok] * wsc;
-              gt *= s;
-              up *= s;
+              const float sc = wgt_sm[c];
+              gt *= sc;
+              up *= sc;
             }
             const float hv = gt / (1.0f + expf(-gt)) * up;
             if (feat < g.I) g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
@@ -331,13 +366,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (FP8) {
-          named_bar_sync(kEpiBar, kEpiThreads);
+          named_bar_sync(bar_id, kEpiThreads);
           for (int c = et; c < BN; c += kEpiThreads) {
             const float m = fmaxf(fmaxf(amax_part[c], amax_part[BN + c]),
                                   fmaxf(amax_part[2 * BN + c], amax_part[3 * BN + c]));
             g.h_amax[static_cast<size_t>(mt) * g.rows_cap + blk * BN + c] = m;
           }
-          named_bar_sync(kEpiBar, kEpiThreads);
         }
       } else {
         const int n = mt * kTileM + 32 * q + lane;  // output feature
@@ -353,20 +387,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int r = blk * BN + c0 + i;
-            int f, t;
-            if (!g.sorted_ids) {
-              f = r;
-              t = r;
-              if (r >= g.T) continue;
-            } else {
-              f = g.sorted_ids[r];
-              if (f < 0 || f >= slots) continue;
-              t = f / g.top_k;
-            }
-            const float wt = load_weight(g.weights, g.weights_dtype, f);
-            const float val = v[i] * wt;
-            if (!nvalid) continue;
+            const int t = tok_sm[c0 + i];
+            if (t < 0 || !nvalid) continue;
+            const float val = v[i] * wgt_sm[c0 + i];
             const size_t o = static_cast<size_t>(t) * g.H + n;
             if (g.top_k == 1) {
               float y = val;
@@ -378,42 +401,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (g.top_k > 1) {
-          // Arrival count per (token, weight tile): the epilogue that brings
-          // the k-th slot finalises the token's 128 outputs of this tile.
-          __threadfence();
-          named_bar_sync(kEpiBar, kEpiThreads);
+          // Arrival count per (token, weight tile). The group barrier orders
+          // every thread's red.add before the counter update, whose release
+          // publishes them; the epilogue that brings a token's k-th slot
+          // acquires all k contributions and finalises the 128 outputs.
+          named_bar_sync(bar_id, kEpiThreads);
           for (int c = et; c < BN; c += kEpiThreads) {
-            const int f = g.sorted_ids[blk * BN + c];
+            const int t = tok_sm[c];
             int flag = 0;
-            if (f >= 0 && f < slots) {
-              int* cnt = g.counters + static_cast<size_t>(f / g.top_k) * g.n_mt + mt;
-              __threadfence();
-              if (atomicAdd(cnt, 1) == g.top_k - 1) {
+            if (t >= 0) {
+              int* cnt = g.counters + static_cast<size_t>(t) * g.n_mt + mt;
+              if (atom_add_acq_rel_gpu(cnt, 1) == g.top_k - 1) {
                 flag = 1;
                 *cnt = 0;
               }
             }
             last_sm[c] = flag;
           }
-          named_bar_sync(kEpiBar, kEpiThreads);
-          __threadfence();
-          for (int c = 0; c < BN; ++c) {
-            if (!last_sm[c]) continue;
-            const int t = g.sorted_ids[blk * BN + c] / g.top_k;
-            if (nvalid) {
-              const size_t o = static_cast<size_t>(t) * g.H + n;
+          named_bar_sync(bar_id, kEpiThreads);
+          if (nvalid) {
+            for (int c = 0; c < BN; ++c) {
+              if (!last_sm[c]) continue;
+              const size_t o = static_cast<size_t>(tok_sm[c]) * g.H + n;
               float y = atomicExch(g.ws + o, 0.0f);
               if (g.addend) y += __bfloat162float(g.addend[o]);
               g.out[o] = __float2bfloat16_rn(y);
             }
           }
-          named_bar_sync(kEpiBar, kEpiThreads);
         }
       }
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
+      named_bar_sync(bar_id, kEpiThreads);  // metadata of this tile no longer read
     }
   }
 

@@ -112,7 +112,7 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
   }
   int grid = max_tiles < num_sms() ? max_tiles : num_sms();
   if (grid < 1) grid = 1;
-  kern<<<grid, moe::kGemmThreads, L::kBytes, s>>>(ta, tb, g);
+  kern<<<grid, moe::EpiCfg<BN>::kThreads, L::kBytes, s>>>(ta, tb, g);
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }

@@ -37,7 +37,7 @@ def bf16_ulp(v):
     return np.ldexp(1.0, (e - 1 - 7).astype(np.int32))
 
 
-def assert_close_rms(out, ref, tol, what="", rounded=None, exact_frac=None):
+def assert_close_rms(out, ref, tol, what="", rounded=None, exact_frac=None, mean_check=True):
     """Tolerance of the layer's float outputs.
 
     The stated bound max|out - ref| <= tol * rms(ref) applies to the arithmetic.
@@ -45,7 +45,9 @@ def assert_close_rms(out, ref, tol, what="", rounded=None, exact_frac=None):
     values that differ only in their last fp32 bits can land one bf16 step
     apart, so each element may also differ by one bf16 ulp of every rounded
     quantity listed in ``rounded`` (default: ``ref`` itself). Two checks guard
-    against errors hiding in that allowance: mean|err| <= tol/10 * rms(ref) and,
+    against errors hiding in that allowance: mean|err| <= tol/10 * rms(ref)
+    (skipped with ``mean_check=False`` where ``ref`` itself carries an extra
+    rounding by construction) and,
     when ``exact_frac`` is given, at least that fraction of the elements equal
     the oracle's bit for bit.
     Returns max|err| / rms(ref).
@@ -60,7 +62,8 @@ def assert_close_rms(out, ref, tol, what="", rounded=None, exact_frac=None):
     bad = err > bound
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond tol*rms + rounding; worst err "
                            f"{err.max():.3e}, rms {rms:.3e}")
-    assert err.mean() <= 0.1 * tol * rms, f"{what}: mean|err| {err.mean():.3e} vs rms {rms:.3e}"
+    if mean_check:
+        assert err.mean() <= 0.1 * tol * rms, f"{what}: mean|err| {err.mean():.3e} vs rms {rms:.3e}"
     if exact_frac is not None:
         frac = float(np.mean(out == ref))
         assert frac >= exact_frac, f"{what}: only {frac:.3f} of the outputs bit-identical"

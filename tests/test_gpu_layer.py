@@ -102,7 +102,7 @@ def test_addend_in_epilogue_equals_separate_add(cuda_lib):
     # fused rounds (addend + routed sum) once; the separate path rounded the
     # routed sum first: one bf16 step of each may separate them
     assert_close_rms(fused.cpu().numpy(), routed + addend, BF16_TOL, "fused vs separate",
-                     rounded=[routed + addend, routed])
+                     rounded=[routed + addend, routed], mean_check=False)
 
 
 def test_rsf_fold_scales_routed_output(cuda_lib):
@@ -115,7 +115,8 @@ def test_rsf_fold_scales_routed_output(cuda_lib):
         layer.routed(torch.cuda.current_stream(), addend=False)
         torch.cuda.synchronize()
         outs.append(layer.out.float().cpu().numpy())
-    assert_close_rms(outs[1], 2.5 * outs[0], BF16_TOL, "rsf fold", rounded=[outs[1], 2.5 * outs[0]])
+    assert_close_rms(outs[1], 2.5 * outs[0], BF16_TOL, "rsf fold", rounded=[outs[1], 2.5 * outs[0]],
+                     mean_check=False)
 
 
 def test_cuda_graph_replay(cuda_lib):
