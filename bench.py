@@ -69,10 +69,13 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+GEMM_SOURCES = ("gemm.cuh", "ptx.cuh")  # the grouped-GEMM kernel's own sources
+
+
 def src_hash() -> str:
     h = hashlib.sha256()
     d = os.path.join(ROOT, "routed_shared_experts_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in GEMM_SOURCES:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
