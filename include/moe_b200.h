@@ -63,6 +63,7 @@ typedef int moe_status_t;
 #define MOE_ERR_SHAPE (-4)             /* sizes the kernels do not cover */
 #define MOE_ERR_CUDA (-5)              /* a CUDA runtime / driver call failed */
 #define MOE_ERR_DEVICE (-6)            /* device error word was set (moe_device_error) */
+#define MOE_ERR_WORKSPACE_LIMIT (-7)   /* problem larger than the library's static workspace */
 
 /* Operand formats. */
 #define MOE_DT_BF16 0
@@ -218,6 +219,43 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h
                                         int T, int top_k, int H, int I, int E, int block_m,
                                         const void* addend, moe_event_t addend_ready, void* acc_ws,
                                         void* out, moe_stream_t stream);
+
+/* Size of the stage-2 workspace that the library itself holds in device memory
+ * for moe_stage2_gemm_accumulate_static_ws (8 MiB on every GPU that loads the
+ * library, kept until the process exits). */
+#define MOE_STAGE2_STATIC_WS_BYTES (8u << 20)
+
+/* moe_stage2_gemm_accumulate_static_ws: moe_stage2_gemm_accumulate for callers
+ * that cannot allocate device memory themselves - plugin interfaces that hand
+ * the operator only its input and output buffers, or processes whose device
+ * memory has already been handed to another allocator's pool, where a
+ * cudaMalloc would fail or could synchronise the device. There is no
+ * counterpart of this call in the pages; it exists for those callers.
+ *
+ * Arguments and results are those of moe_stage2_gemm_accumulate without
+ * acc_ws. In its place the library uses a statically allocated device array of
+ * MOE_STAGE2_STATIC_WS_BYTES. This call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *   - Limit: top_k > 1 needs moe_stage2_workspace_bytes(T, H) <=
+ *     MOE_STAGE2_STATIC_WS_BYTES (for H = 2048 up to T = 1016); larger
+ *     problems return MOE_ERR_WORKSPACE_LIMIT (message in
+ *     moe_last_cuda_error()) and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - The array is shared by every call on a device and keeps the last call's
+ *     contents; each call clears the part it uses on `stream` before its
+ *     kernel. Calls whose work overlaps on the GPU (concurrent streams) race
+ *     on the array: serialise them. */
+moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const float* h_amax,
+                                                  const void* w2, const float* w2_scale,
+                                                  const void* weights, int weights_dtype,
+                                                  const int32_t* sorted_ids,
+                                                  const int32_t* block_expert,
+                                                  const int32_t* num_padded, int T, int top_k,
+                                                  int H, int I, int E, int block_m,
+                                                  const void* addend, moe_event_t addend_ready,
+                                                  void* out, moe_stream_t stream);
 
 /* shared_expert_gate_dot: out[t] = sigmoid(sum_k x[t,k] * w[k]) ([56789]),
  * one fused kernel, fp32 accumulation, the result stored in x's dtype (the

@@ -36,6 +36,8 @@ SIGNATURES = {
     "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_stage2_gemm_accumulate": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                         _P, _P, _P]),
+    "moe_stage2_gemm_accumulate_static_ws": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                  _P, _P, _P, _P]),
     "shared_expert_gate_dot": (_I, [_I, _P, _P, _I, _I, _I, _P, _P]),
 }
 
@@ -47,7 +49,7 @@ class MoEError(RuntimeError):
         lib_ = lib()
         msg = lib_.moe_status_string(status).decode()
         cuda = lib_.moe_last_cuda_error().decode()
-        super().__init__(f"{fn}: {msg}" + (f" ({cuda})" if status == -5 and cuda else ""))
+        super().__init__(f"{fn}: {msg}" + (f" ({cuda})" if status in (-5, -7) and cuda else ""))
         self.status = status
 
 
@@ -142,6 +144,17 @@ def moe_stage2_gemm_accumulate(dtype, h, h_amax, w2, w2_scale, weights, weights_
         dtype, _ptr(h), _ptr(h_amax), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
         _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
         _event(addend_ready), _ptr(acc_ws), _ptr(out), _stream(stream)))
+
+
+def moe_stage2_gemm_accumulate_static_ws(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids,
+                                         block_expert, num_padded, T, top_k, H, I, E, block_m, addend,
+                                         addend_ready, out, stream=None):
+    """Stage 2 with the library's own static workspace (no device allocation
+    by the caller or the library); see include/moe_b200.h for its limit."""
+    _check("moe_stage2_gemm_accumulate_static_ws", lib().moe_stage2_gemm_accumulate_static_ws(
+        dtype, _ptr(h), _ptr(h_amax), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
+        _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
+        _event(addend_ready), _ptr(out), _stream(stream)))
 
 
 def shared_expert_gate_dot(dtype, x, w, apply_sigmoid, out, stream=None):

@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "moe_b200.h"
 #include "gate.cuh"
@@ -136,6 +137,30 @@ size_t capacity(int T, int k, int E, int bm) {
   return (n + bm - 1) / bm * bm;
 }
 
+// Stage-2 workspace owned by the library, for callers that cannot allocate
+// (moe_stage2_gemm_accumulate_static_ws). Zero at module load.
+static __device__ __align__(256) unsigned char g_stage2_static_ws[MOE_STAGE2_STATIC_WS_BYTES];
+
+// Device address of g_stage2_static_ws, looked up once per device with that
+// device current. In host code the symbol is only a host-side stand-in.
+std::mutex g_static_ws_mu;
+void* g_static_ws_addr[64];
+
+moe_status_t static_ws_address(void** out) {
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_stage2_static_ws);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(g_stage2_static_ws)");
+    g_static_ws_addr[dev] = p;
+  }
+  *out = g_static_ws_addr[dev];
+  return MOE_OK;
+}
+
 }  // namespace
 
 // ======================================================================== ABI
@@ -151,6 +176,7 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_SHAPE: return "MOE_ERR_SHAPE";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    case MOE_ERR_WORKSPACE_LIMIT: return "MOE_ERR_WORKSPACE_LIMIT";
   }
   return "MOE_ERR_UNKNOWN";
 }
@@ -390,6 +416,43 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
   return launch_gemm<false, false>(block_m, ta, tb, g, max_tiles, s);
+}
+
+moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const float* h_amax, const void* w2,
+                                                  const float* w2_scale, const void* weights, int weights_dtype,
+                                                  const int32_t* sorted_ids, const int32_t* block_expert,
+                                                  const int32_t* num_padded, int T, int top_k, int H, int I, int E,
+                                                  int block_m, const void* addend, moe_event_t addend_ready,
+                                                  void* out, moe_stream_t stream) {
+  // The argument checks of moe_stage2_gemm_accumulate, repeated here so that
+  // nothing (not even the clearing memset) is enqueued for an invalid call.
+  if (dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
+    return MOE_ERR_INVALID_ARG;
+  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
+  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
+  if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
+    return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)))
+    return MOE_ERR_ALIGNMENT;
+  void* ws = nullptr;
+  if (top_k > 1) {
+    const size_t need = moe_stage2_workspace_bytes(T, H);
+    if (need > MOE_STAGE2_STATIC_WS_BYTES) {
+      snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+               "stage-2 workspace of %zu bytes exceeds the static %u bytes (T=%d, H=%d)", need,
+               static_cast<unsigned>(MOE_STAGE2_STATIC_WS_BYTES), T, H);
+      return MOE_ERR_WORKSPACE_LIMIT;
+    }
+    const moe_status_t r = static_ws_address(&ws);
+    if (r != MOE_OK) return r;
+    MOE_CK(cudaMemsetAsync(ws, 0, need, as_stream(stream)));
+  }
+  return moe_stage2_gemm_accumulate(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids,
+                                    block_expert, num_padded, T, top_k, H, I, E, block_m, addend, addend_ready, ws,
+                                    out, stream);
 }
 
 }  // extern "C"
