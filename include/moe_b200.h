@@ -108,9 +108,12 @@ size_t moe_sorted_capacity(int T, int top_k, int E, int block_m);
  * zeroes it ONCE after allocating it; each complete call leaves it zeroed. */
 size_t moe_stage2_workspace_bytes(int T, int H);
 
-/* Bytes of the per-row partial-amax buffer that moe_stage1_gemm writes for
- * MOE_DT_FP8_E4M3 (ceil(I/64) floats per sorted row); 0 for other dtypes. */
-size_t moe_stage1_amax_bytes(int dtype, int rows, int I);
+/* Bytes of the stage-1 workspace for `dtype` (0 when none is needed). For
+ * MOE_DT_FP8_E4M3: the unquantised h as fp32, a per-tile row amax and one
+ * arrival counter per token block, for `capacity` rows of I columns. The
+ * caller zeroes it ONCE after allocating it; each complete call leaves the
+ * counters at zero. */
+size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int I, int block_m);
 
 /* ------------------------------------------------------------------------ */
 
@@ -162,7 +165,9 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
  *     a   = W13[e] . x[t]                           (2I outputs, fp32 accumulate)
  *     a  *= x_scale[t] * w13_scale[e]               (MOE_DT_FP8_E4M3; [6106])
  *     h_r = SiLU(a[0:I]) * a[I:2I]
- * tcgen05 tensor cores, weights streamed by TMA, token rows gathered by TMA.
+ * then h_r is stored in the stage-2 operand format ([6106]: quantisation fused
+ * after the activation). tcgen05 tensor cores, weights streamed by TMA, token
+ * rows gathered by TMA.
  *   dtype      MOE_DT_BF16 or MOE_DT_FP8_E4M3.
  *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8) or NULL.
  *   w13        [E,2I,H]: rows 0..I-1 gate, I..2I-1 up (K = H contiguous);
@@ -172,19 +177,20 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
  *              token r, expert 0, rows padded to a multiple of block_m; used
  *              for the shared expert, E = 1, k = 1); block_expert and
  *              num_padded are then ignored.
- *   h          [capacity rows, I] bf16 (padded rows hold don't-care values).
- *              BF16: the stage-2 operand. FP8: the unquantised h; the e4m3
- *              quantisation (one scale amax/448 per row, [6106] "fused quant")
- *              happens when stage 2 stages the rows for the tensor core.
- *   h_amax     fp32 [ceil(I/64), capacity rows]: FP8 per-tile row amax (NULL
- *              for BF16).
+ *   h          [capacity rows, I] (padded rows hold don't-care values):
+ *              BF16: bf16. FP8: e4m3 codes, row r scaled by h_scale[r].
+ *   h_scale    FP8: fp32 [capacity rows], amax(h_r)/448 (1 for an all-zero
+ *              row); the codes are e4m3(h_r / h_scale[r]), round to nearest
+ *              even, saturating. NULL for BF16.
+ *   ws         FP8: moe_stage1_workspace_bytes(...) bytes, zeroed once by the
+ *              caller. NULL for BF16.
  * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8), I % 64 == 0, block_m in
- * {16,32,64,128,256}, 16-byte aligned x, w13, h. */
-moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, const void* w13,
-                             const float* w13_scale, const int32_t* sorted_ids,
+ * {16,32,64,128,256}, 16-byte aligned x, w13, h, ws. */
+moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, const void* w13,
+                             const void* w13_scale, const int32_t* sorted_ids,
                              const int32_t* block_expert, const int32_t* num_padded, int T,
-                             int top_k, int H, int I, int E, int block_m, void* h, float* h_amax,
-                             moe_stream_t stream);
+                             int top_k, int H, int I, int E, int block_m, void* h, void* h_scale,
+                             void* ws, moe_stream_t stream);
 
 /* moe_stage2_gemm_accumulate: per sorted row r (slot f, token t, expert e):
  *     y_r   = W2[e] . h_r                           (H outputs, fp32 accumulate)
@@ -195,7 +201,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, con
  * commit 2): no separate scale, add or zeroing kernel runs. Partial sums meet
  * in an fp32 workspace; the epilogue that brings a token's last slot adds the
  * addend, rounds once to bf16, writes out and re-zeroes its workspace slice.
- *   dtype       as stage 1; h / h_amax are stage 1's outputs.
+ *   dtype       as stage 1; h / h_scale are stage 1's outputs.
  *   w2          [E,H,I] (K = I contiguous); w2_scale fp32 [E] (FP8) or NULL.
  *   weights     [T*k] per slot f (routing weights, scale folded in), dtype
  *               weights_dtype = MOE_DT_F32, or MOE_DT_BF16 / MOE_DT_FP16 (the
@@ -210,10 +216,10 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, con
  * Identity routing (sorted_ids == NULL): as in stage 1; with top_k == 1 each
  * row's result goes straight to out (this is how the shared expert's output
  * becomes the addend of the routed call).
- * Checks: H % 16 == 0, I % 64 == 0 (bf16) / % 128 == 0 (fp8), block_m as
- * stage 1, 16-byte aligned h, w2, out, addend. */
-moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h_amax,
-                                        const void* w2, const float* w2_scale, const void* weights,
+ * Checks: H % 128 == 0, I % 64 == 0, block_m as stage 1, 16-byte aligned h,
+ * w2, out, addend, acc_ws. */
+moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale,
+                                        const void* w2, const void* w2_scale, const void* weights,
                                         int weights_dtype, const int32_t* sorted_ids,
                                         const int32_t* block_expert, const int32_t* num_padded,
                                         int T, int top_k, int H, int I, int E, int block_m,
@@ -247,8 +253,8 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h
  *     contents; each call clears the part it uses on `stream` before its
  *     kernel. Calls whose work overlaps on the GPU (concurrent streams) race
  *     on the array: serialise them. */
-moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const float* h_amax,
-                                                  const void* w2, const float* w2_scale,
+moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const void* h_scale,
+                                                  const void* w2, const void* w2_scale,
                                                   const void* weights, int weights_dtype,
                                                   const int32_t* sorted_ids,
                                                   const int32_t* block_expert,

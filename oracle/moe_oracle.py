@@ -201,17 +201,35 @@ def sigmoid_fp32(logits) -> np.ndarray:
     return fp32_round(1.0 / (1.0 + np.exp(-l)))
 
 
-def sigmoid_fp32_hazards(logits, margin_log2: int = -44) -> int:
-    """Count scores whose float64 sigmoid lies so close to an fp32 rounding
-    midpoint (relative distance < 2**margin_log2) that an exp differing by a few
-    float64 ulps could round to the other fp32 neighbour."""
+def sigmoid_fp32_hazard_mask(logits, margin_log2: int = -46) -> np.ndarray:
+    """Scores whose float64 sigmoid lies within 2**margin_log2 (relative) of an
+    fp32 rounding midpoint. Two correct evaluations of 1/(1+exp(-l)) in float64
+    (exp within a few ulps, then one add and one divide) differ by well under
+    2**-48 relative, so only these scores can round to different fp32 values
+    on two machines."""
     l = np.asarray(logits, dtype=np.float32).astype(np.float64)
     v = 1.0 / (1.0 + np.exp(-l))
     r = fp32_round(v)
     _, e = np.frexp(r)
     half_ulp = np.ldexp(1.0, (e.astype(np.int64) - 1 - 24).astype(np.int32))
     mid = np.where(v >= r, r + half_ulp, r - half_ulp)
-    return int(np.count_nonzero(np.abs(v - mid) < np.abs(v) * 2.0**margin_log2))
+    return np.abs(v - mid) < np.abs(v) * 2.0**margin_log2
+
+
+def sigmoid_fp32_hazards(logits, margin_log2: int = -46) -> int:
+    """Number of scores flagged by ``sigmoid_fp32_hazard_mask``."""
+    return int(np.count_nonzero(sigmoid_fp32_hazard_mask(logits, margin_log2)))
+
+
+def sigmoid_fp32_other(logits) -> np.ndarray:
+    """The fp32 neighbour of the float64 sigmoid on the other side of it from
+    ``sigmoid_fp32`` (the rounding another machine may take at a hazard)."""
+    l = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    v = 1.0 / (1.0 + np.exp(-l))
+    r = sigmoid_fp32(logits).astype(np.float32)
+    up = np.nextafter(r, np.float32(np.inf))
+    dn = np.nextafter(r, np.float32(-np.inf))
+    return np.where(v >= r.astype(np.float64), up, dn).astype(np.float64)
 
 
 def router_grouped_sigmoid_topk(
@@ -222,6 +240,7 @@ def router_grouped_sigmoid_topk(
     topk_group: int,
     renormalize: bool = True,
     rsf: float = 1.0,
+    scores=None,
 ):
     """Biased grouped sigmoid top-k (the ``biased_grouped_topk`` of vllm PR
     65207, "Purpose", commit 1), with the usual reading of its steps:
@@ -234,11 +253,13 @@ def router_grouped_sigmoid_topk(
     5. among experts of kept groups pick k by (c desc, index asc);
     6. weights use the unbiased scores: s_j / sum_sel s * rsf (renormalize) or
        s_j * rsf — the scale is applied here, inside top-k.
+    ``scores`` replaces step 1 with given fp32 scores (used to evaluate the
+    other rounding of a hazard score).
     """
     l = np.asarray(logits, dtype=np.float32)
     T, E = l.shape
     gsize = E // n_group
-    s = sigmoid_fp32(l).astype(np.float32)
+    s = (sigmoid_fp32(l) if scores is None else np.asarray(scores, np.float64)).astype(np.float32)
     b = np.zeros(E, np.float32) if correction_bias is None else np.asarray(correction_bias, np.float32)
     c = (s + b[None, :]).astype(np.float32)  # IEEE fp32 addition
     ids = np.empty((T, top_k), np.int32)

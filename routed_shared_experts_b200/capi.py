@@ -30,10 +30,10 @@ SIGNATURES = {
     "moe_device_error": (_I, [ctypes.POINTER(ctypes.c_int), _P]),
     "moe_sorted_capacity": (_SZ, [_I, _I, _I, _I]),
     "moe_stage2_workspace_bytes": (_SZ, [_I, _I]),
-    "moe_stage1_amax_bytes": (_SZ, [_I, _I, _I]),
+    "moe_stage1_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "moe_router_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "moe_align_sort": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
-    "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_stage2_gemm_accumulate": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                         _P, _P, _P]),
     "moe_stage2_gemm_accumulate_static_ws": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I,
@@ -104,8 +104,8 @@ def stage2_workspace_bytes(T: int, H: int) -> int:
     return lib().moe_stage2_workspace_bytes(T, H)
 
 
-def stage1_amax_bytes(dtype: int, rows: int, I: int) -> int:
-    return lib().moe_stage1_amax_bytes(dtype, rows, I)
+def stage1_workspace_bytes(dtype: int, T: int, top_k: int, E: int, I: int, block_m: int) -> int:
+    return lib().moe_stage1_workspace_bytes(dtype, T, top_k, E, I, block_m)
 
 
 def device_error(stream=None) -> int:
@@ -131,28 +131,28 @@ def moe_align_sort(topk_ids, E, block_m, sorted_ids, block_expert, expert_counts
 
 
 def moe_stage1_gemm(dtype, x, x_scale, w13, w13_scale, sorted_ids, block_expert, num_padded, T, top_k, H, I, E,
-                    block_m, h, h_amax, stream=None):
+                    block_m, h, h_scale, ws, stream=None):
     _check("moe_stage1_gemm", lib().moe_stage1_gemm(
         dtype, _ptr(x), _ptr(x_scale), _ptr(w13), _ptr(w13_scale), _ptr(sorted_ids), _ptr(block_expert),
-        _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(h), _ptr(h_amax), _stream(stream)))
+        _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(h), _ptr(h_scale), _ptr(ws), _stream(stream)))
 
 
-def moe_stage2_gemm_accumulate(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids, block_expert,
+def moe_stage2_gemm_accumulate(dtype, h, h_scale, w2, w2_scale, weights, weights_dtype, sorted_ids, block_expert,
                                num_padded, T, top_k, H, I, E, block_m, addend, addend_ready, acc_ws, out,
                                stream=None):
     _check("moe_stage2_gemm_accumulate", lib().moe_stage2_gemm_accumulate(
-        dtype, _ptr(h), _ptr(h_amax), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
+        dtype, _ptr(h), _ptr(h_scale), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
         _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
         _event(addend_ready), _ptr(acc_ws), _ptr(out), _stream(stream)))
 
 
-def moe_stage2_gemm_accumulate_static_ws(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids,
+def moe_stage2_gemm_accumulate_static_ws(dtype, h, h_scale, w2, w2_scale, weights, weights_dtype, sorted_ids,
                                          block_expert, num_padded, T, top_k, H, I, E, block_m, addend,
                                          addend_ready, out, stream=None):
     """Stage 2 with the library's own static workspace (no device allocation
     by the caller or the library); see include/moe_b200.h for its limit."""
     _check("moe_stage2_gemm_accumulate_static_ws", lib().moe_stage2_gemm_accumulate_static_ws(
-        dtype, _ptr(h), _ptr(h_amax), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
+        dtype, _ptr(h), _ptr(h_scale), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
         _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
         _event(addend_ready), _ptr(out), _stream(stream)))
 

@@ -54,14 +54,17 @@ struct GemmArgs {
   int n_mt;    // weight tiles per token block
   int num_kb;  // K stages per tile
   // stage 1 outputs
-  __nv_bfloat16* h;  // [rows, I]
-  float* h_amax;     // fp8: [ceil(I/64)][rows_cap]
+  __nv_bfloat16* h;  // bf16: h [rows, I]
+  float* h32;        // fp8: the unquantised h [rows, I] in fp32 (workspace)
+  float* h_amax;     // fp8: per-tile row amax [n_mt][rows_cap] (workspace)
+  int* blk_cnt;      // fp8: finished weight tiles per token block (workspace, self-cleaning)
+  uint8_t* hq;       // fp8: e4m3 codes of h [rows, I]
   int rows_cap;
   const float* x_scale;  // fp8: [T]
-  const float* w_scale;  // fp8: [E]
+  const float* w_scale;  // fp8: [E] (stage 1: W13, stage 2: W2)
+  // stage 1 output / stage 2 input: fp8 per-row scale of h [rows]
+  float* h_scale;
   // stage 2
-  const float* h_amax_in;  // fp8: stage-1 partial amax
-  int n_amax_tiles;
   const void* weights;  // [T*k] or nullptr
   int weights_dtype;    // 4 = f32, 0 = bf16, 1 = fp16
   const __nv_bfloat16* addend;
@@ -113,6 +116,43 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
   int old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+
+// e4m3 with round-to-nearest-even and saturation to +-448 (two values).
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Quantise the BN rows of token block `blk` from the unquantised fp32 h to
+// e4m3 with one fp32 scale per row, s = amax / 448 (amax = 0 -> s = 1), code =
+// e4m3(h / s) (round to nearest even, saturating). Run by one epilogue
+// warpgroup (128 threads, named barrier `bar_id`) after it has acquired every
+// weight tile of the block; `scale_sm` is BN floats of its shared memory.
+template <int BN>
+__device__ __noinline__ void quantize_block_rows(const GemmArgs& g, int blk, int et, int bar_id, float* scale_sm) {
+  for (int c = et; c < BN; c += kEpiThreads) {
+    const int r = blk * BN + c;
+    float m = 0.f;
+    for (int t = 0; t < g.n_mt; ++t) m = fmaxf(m, __ldcg(g.h_amax + static_cast<size_t>(t) * g.rows_cap + r));
+    const float sc = m > 0.f ? m / 448.0f : 1.0f;
+    scale_sm[c] = sc;
+    g.h_scale[r] = sc;
+  }
+  named_bar_sync(bar_id, kEpiThreads);
+  const int chunks = g.I / 8;  // 8 columns per step: two 16-byte fp32 loads, one 8-byte e4m3 store
+  const int total = BN * chunks;
+  for (int i = et; i < total; i += kEpiThreads) {
+    const int c = i / chunks;
+    const size_t off = static_cast<size_t>(blk * BN + c) * g.I + static_cast<size_t>(i - c * chunks) * 8;
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(g.h32 + off));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(g.h32 + off + 4));
+    const float sc = scale_sm[c];
+    const uint32_t q0 = cvt_e4m3x2(a.x / sc, a.y / sc), q1 = cvt_e4m3x2(a.z / sc, a.w / sc);
+    const uint32_t q2 = cvt_e4m3x2(b.x / sc, b.y / sc), q3 = cvt_e4m3x2(b.z / sc, b.w / sc);
+    *reinterpret_cast<uint2*>(g.hq + off) = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
+  }
 }
 
 template <int BN, int STAGES, bool S1, bool FP8>
@@ -289,7 +329,8 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
     int* gsm = group_base + grp * L::kGroupWords;
     volatile int* ok_sm = gsm;
     int* tok_sm = gsm + 4;                        // token of each column, -1 = padding
-    float* wgt_sm = reinterpret_cast<float*>(tok_sm + BN);  // stage 2: top-k weight; stage 1 fp8: x scale
+    float* wgt_sm = reinterpret_cast<float*>(tok_sm + BN);  // per-column factor: stage 1 fp8 x and W13 scales;
+                                                            // stage 2 top-k weight (x h and W2 scales for fp8)
     int* last_sm = reinterpret_cast<int*>(wgt_sm + BN);
     float* amax_part = reinterpret_cast<float*>(last_sm + BN);
     int j = 0;
@@ -315,7 +356,7 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
         float w = 0.f;
         if (t >= 0) {
           if (S1) w = FP8 ? g.x_scale[t] * g.w_scale[expert] : 1.0f;
-          else w = load_weight(g.weights, g.weights_dtype, f);
+          else w = load_weight(g.weights, g.weights_dtype, f) * (FP8 ? g.h_scale[r] * g.w_scale[expert] : 1.0f);
         }
         wgt_sm[c] = w;
       }
@@ -353,7 +394,10 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
               up *= sc;
             }
             const float hv = gt / (1.0f + expf(-gt)) * up;
-            if (feat < g.I) g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
+            if (feat < g.I) {
+              if (FP8) g.h32[static_cast<size_t>(r) * g.I + feat] = hv;
+              else g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
+            }
             if (FP8) {
               // per-row amax of this tile's 16 features of the half-warp
               float m = fabsf(hv);
@@ -372,6 +416,21 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
                                   fmaxf(amax_part[2 * BN + c], amax_part[3 * BN + c]));
             g.h_amax[static_cast<size_t>(mt) * g.rows_cap + blk * BN + c] = m;
           }
+          // The group that finishes the last weight tile of this token block
+          // quantises the block's rows: one scale amax/448 per row over all I
+          // columns (ROCm/aiter PR 6106, "Technical Details": quantisation
+          // fused after the activation). The barrier orders this group's h and
+          // amax stores before the counter's release; the acquire of the last
+          // arrival makes every tile's stores visible.
+          named_bar_sync(bar_id, kEpiThreads);
+          if (et == 0) {
+            int* cnt = g.blk_cnt + blk;
+            const bool last = atom_add_acq_rel_gpu(cnt, 1) == g.n_mt - 1;
+            if (last) *cnt = 0;
+            last_sm[0] = last ? 1 : 0;
+          }
+          named_bar_sync(bar_id, kEpiThreads);
+          if (last_sm[0]) quantize_block_rows<BN>(g, blk, et, bar_id, amax_part);
         }
       } else {
         const int n = mt * kTileM + 32 * q + lane;  // output feature

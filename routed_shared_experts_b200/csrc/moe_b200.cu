@@ -137,6 +137,18 @@ size_t capacity(int T, int k, int E, int bm) {
   return (n + bm - 1) / bm * bm;
 }
 
+// Stage-1 workspace of the fp8 path: unquantised fp32 h [rows, I], per-tile
+// row amax [I/64][rows], one arrival counter per token block; 256-byte aligned parts.
+struct Stage1Ws {
+  size_t amax_off, cnt_off, total;
+  Stage1Ws(size_t rows, int I, int bm) {
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    amax_off = up(rows * static_cast<size_t>(I) * 4);
+    cnt_off = amax_off + up(static_cast<size_t>((I + 63) / 64) * rows * 4);
+    total = cnt_off + up(rows / bm * 4);
+  }
+};
+
 // Stage-2 workspace owned by the library, for callers that cannot allocate
 // (moe_stage2_gemm_accumulate_static_ws). Zero at module load.
 static __device__ __align__(256) unsigned char g_stage2_static_ws[MOE_STAGE2_STATIC_WS_BYTES];
@@ -209,9 +221,9 @@ size_t moe_stage2_workspace_bytes(int T, int H) {
   return static_cast<size_t>(T) * H * sizeof(float) + static_cast<size_t>(T) * n_mt * sizeof(int);
 }
 
-size_t moe_stage1_amax_bytes(int dtype, int rows, int I) {
-  if (dtype != MOE_DT_FP8_E4M3 || rows < 1 || I < 1) return 0;
-  return static_cast<size_t>((I + 63) / 64) * rows * sizeof(float);
+size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int I, int block_m) {
+  if (dtype != MOE_DT_FP8_E4M3 || T < 1 || top_k < 1 || E < 1 || I < 1 || !valid_block_m(block_m)) return 0;
+  return Stage1Ws(capacity(T, top_k, E, block_m), I, block_m).total;
 }
 
 moe_status_t moe_router_topk(const float* logits, const float* correction_bias, int T, int E, int top_k, int mode,
@@ -285,10 +297,10 @@ moe_status_t shared_expert_gate_dot(int dtype, const void* x, const void* w, int
   return MOE_OK;
 }
 
-moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, const void* w13,
-                             const float* w13_scale, const int32_t* sorted_ids, const int32_t* block_expert,
-                             const int32_t* num_padded, int T, int top_k, int H, int I, int E, int block_m, void* h,
-                             float* h_amax, moe_stream_t stream) {
+moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, const void* w13, const void* w13_scale,
+                             const int32_t* sorted_ids, const int32_t* block_expert, const int32_t* num_padded, int T,
+                             int top_k, int H, int I, int E, int block_m, void* h, void* h_scale, void* ws,
+                             moe_stream_t stream) {
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
   if (dtype != MOE_DT_BF16 && !fp8) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!x || !w13 || !h) return MOE_ERR_INVALID_ARG;
@@ -296,15 +308,14 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, con
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  if (fp8 && (!x_scale || !w13_scale || !h_amax)) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!x_scale || !w13_scale || !h_scale || !ws)) return MOE_ERR_INVALID_ARG;
   if (H % (fp8 ? 128 : 64) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(w13) || !aligned16(h)) return MOE_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(h) || (ws && !aligned16(ws))) return MOE_ERR_ALIGNMENT;
 
   const int es = fp8 ? 1 : 2;
   const int ke = fp8 ? 128 : 64;
-  const size_t rows_cap = sorted_ids ? capacity(T, top_k, E, block_m)
-                                     : static_cast<size_t>((T + block_m - 1) / block_m) * block_m;
-  const int cap_blocks = static_cast<int>((rows_cap + block_m - 1) / block_m);
+  const size_t rows_cap = capacity(T, top_k, E, block_m);  // identity routing: T rounded up to block_m
+  const int cap_blocks = static_cast<int>(rows_cap / block_m);
   const CUtensorMapDataType tdt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 
   // W13 as 5-D (K, row-in-16, gate|up, 16-row group, expert): one box brings
@@ -339,32 +350,41 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const float* x_scale, con
   g.I = I;
   g.n_mt = I / 64;
   g.num_kb = H / ke;
-  g.h = static_cast<__nv_bfloat16*>(h);
-  g.h_amax = h_amax;
   g.rows_cap = static_cast<int>(rows_cap);
-  g.x_scale = x_scale;
-  g.w_scale = w13_scale;
+  if (fp8) {
+    const Stage1Ws L(rows_cap, I, block_m);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    g.h32 = reinterpret_cast<float*>(w);
+    g.h_amax = reinterpret_cast<float*>(w + L.amax_off);
+    g.blk_cnt = reinterpret_cast<int*>(w + L.cnt_off);
+    g.hq = static_cast<uint8_t*>(h);
+    g.h_scale = static_cast<float*>(h_scale);
+    g.x_scale = static_cast<const float*>(x_scale);
+    g.w_scale = static_cast<const float*>(w13_scale);
+  } else {
+    g.h = static_cast<__nv_bfloat16*>(h);
+  }
   const int max_tiles = cap_blocks * g.n_mt;
   cudaStream_t s = as_stream(stream);
   return fp8 ? launch_gemm<true, true>(block_m, ta, tb, g, max_tiles, s)
              : launch_gemm<true, false>(block_m, ta, tb, g, max_tiles, s);
 }
 
-moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h_amax, const void* w2,
-                                        const float* w2_scale, const void* weights, int weights_dtype,
+moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale, const void* w2,
+                                        const void* w2_scale, const void* weights, int weights_dtype,
                                         const int32_t* sorted_ids, const int32_t* block_expert,
                                         const int32_t* num_padded, int T, int top_k, int H, int I, int E,
                                         int block_m, const void* addend, moe_event_t addend_ready, void* acc_ws,
                                         void* out, moe_stream_t stream) {
-  if (dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
-  (void)h_amax;
-  (void)w2_scale;
+  const bool fp8 = dtype == MOE_DT_FP8_E4M3;
+  if (dtype != MOE_DT_BF16 && !fp8) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
   if (top_k > 1 && !acc_ws) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
   if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
     return MOE_ERR_UNSUPPORTED_DTYPE;
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
@@ -372,25 +392,25 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h
       (acc_ws && !aligned16(acc_ws)))
     return MOE_ERR_ALIGNMENT;
 
-  const int es = 2;
-  const int ke = 64;
-  const size_t rows_cap = sorted_ids ? capacity(T, top_k, E, block_m)
-                                     : static_cast<size_t>((T + block_m - 1) / block_m) * block_m;
-  const int cap_blocks = static_cast<int>((rows_cap + block_m - 1) / block_m);
+  const int es = fp8 ? 1 : 2;
+  const int ke = fp8 ? 128 : 64;
+  const size_t rows_cap = capacity(T, top_k, E, block_m);
+  const int cap_blocks = static_cast<int>(rows_cap / block_m);
+  const CUtensorMapDataType tdt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap ta, tb;
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(E)};
     const cuuint64_t st[2] = {static_cast<cuuint64_t>(I) * es, static_cast<cuuint64_t>(H) * I * es};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(moe::kTileM), 1};
-    moe_status_t r = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w2, dims, st, box);
+    moe_status_t r = make_map(&ta, tdt, 3, w2, dims, st, box);
     if (r != MOE_OK) return r;
   }
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(cap_blocks) * block_m};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(rows_cap)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(I) * es};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
-    moe_status_t r = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h, dims, st, box);
+    moe_status_t r = make_map(&tb, tdt, 2, h, dims, st, box);
     if (r != MOE_OK) return r;
   }
   cudaStream_t s = as_stream(stream);
@@ -407,31 +427,36 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const float* h
   g.H = H;
   g.I = I;
   g.n_mt = H / moe::kTileM;
-  g.num_kb = I / ke;
+  g.num_kb = (I + ke - 1) / ke;
+  g.rows_cap = static_cast<int>(rows_cap);
   g.weights = weights;
   g.weights_dtype = weights_dtype;
+  g.h_scale = fp8 ? const_cast<float*>(static_cast<const float*>(h_scale)) : nullptr;
+  g.w_scale = fp8 ? static_cast<const float*>(w2_scale) : nullptr;
   g.addend = static_cast<const __nv_bfloat16*>(addend);
   g.ws = static_cast<float*>(acc_ws);
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
-  return launch_gemm<false, false>(block_m, ta, tb, g, max_tiles, s);
+  return fp8 ? launch_gemm<false, true>(block_m, ta, tb, g, max_tiles, s)
+             : launch_gemm<false, false>(block_m, ta, tb, g, max_tiles, s);
 }
 
-moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const float* h_amax, const void* w2,
-                                                  const float* w2_scale, const void* weights, int weights_dtype,
+moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const void* h_scale, const void* w2,
+                                                  const void* w2_scale, const void* weights, int weights_dtype,
                                                   const int32_t* sorted_ids, const int32_t* block_expert,
                                                   const int32_t* num_padded, int T, int top_k, int H, int I, int E,
                                                   int block_m, const void* addend, moe_event_t addend_ready,
                                                   void* out, moe_stream_t stream) {
   // The argument checks of moe_stage2_gemm_accumulate, repeated here so that
   // nothing (not even the clearing memset) is enqueued for an invalid call.
-  if (dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_DT_FP8_E4M3 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
   if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
     return MOE_ERR_UNSUPPORTED_DTYPE;
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
@@ -450,7 +475,7 @@ moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, cons
     if (r != MOE_OK) return r;
     MOE_CK(cudaMemsetAsync(ws, 0, need, as_stream(stream)));
   }
-  return moe_stage2_gemm_accumulate(dtype, h, h_amax, w2, w2_scale, weights, weights_dtype, sorted_ids,
+  return moe_stage2_gemm_accumulate(dtype, h, h_scale, w2, w2_scale, weights, weights_dtype, sorted_ids,
                                     block_expert, num_padded, T, top_k, H, I, E, block_m, addend, addend_ready, ws,
                                     out, stream);
 }

@@ -47,12 +47,17 @@ class MoELayer:
         self.expert_counts = torch.empty(E, **i32)
         self.expert_offsets = torch.empty(E + 1, **i32)
         self.num_padded = torch.empty(1, **i32)
-        self.h = torch.empty((cap, I), dtype=torch.bfloat16, device=dev)
-        self.h_s = torch.empty((cap_s, Is), dtype=torch.bfloat16, device=dev)
-        amax_b = capi.stage1_amax_bytes(self.dt, cap, I)
-        amax_bs = capi.stage1_amax_bytes(self.dt, cap_s, Is)
-        self.h_amax = torch.empty(max(amax_b // 4, 1), dtype=torch.float32, device=dev) if amax_b else None
-        self.h_amax_s = torch.empty(max(amax_bs // 4, 1), dtype=torch.float32, device=dev) if amax_bs else None
+        # stage-1 output h in the stage-2 operand format (+ per-row scales for fp8)
+        hdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.uint8
+        self.h = torch.empty((cap, I), dtype=hdt, device=dev)
+        self.h_s = torch.empty((cap_s, Is), dtype=hdt, device=dev)
+        fp8 = cfg.dtype == "fp8"
+        self.h_scale = torch.empty(cap, dtype=torch.float32, device=dev) if fp8 else None
+        self.h_scale_s = torch.empty(cap_s, dtype=torch.float32, device=dev) if fp8 else None
+        ws1 = capi.stage1_workspace_bytes(self.dt, T, k, E, I, bm)
+        ws1s = capi.stage1_workspace_bytes(self.dt, T, 1, 1, Is, bm)
+        self.ws1 = torch.zeros(ws1, dtype=torch.uint8, device=dev) if ws1 else None  # zeroed once
+        self.ws1_s = torch.zeros(ws1s, dtype=torch.uint8, device=dev) if ws1s else None
         gdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float16
         self.gate = torch.empty(T, dtype=gdt, device=dev) if cfg.shared_gate else None
         self.addend = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -71,9 +76,9 @@ class MoELayer:
         if self.gate is not None:
             capi.shared_expert_gate_dot(capi.MOE_DT_BF16, inp["x"], inp["w_gate"], True, self.gate, stream)
         capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13s"], inp.get("w13s_scale"),
-                             None, None, None, T, 1, H, Is, 1, self.bm, self.h_s, self.h_amax_s, stream)
+                             None, None, None, T, 1, H, Is, 1, self.bm, self.h_s, self.h_scale_s, self.ws1_s, stream)
         wdt = capi.MOE_DT_BF16 if self.gate is not None else capi.MOE_DT_F32
-        capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_amax_s, inp["w2s"], inp.get("w2s_scale"),
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_scale_s, inp["w2s"], inp.get("w2s_scale"),
                                         self.gate, wdt, None, None, None, T, 1, H, Is, 1, self.bm, None, None,
                                         None, self.addend, stream)
 
@@ -91,13 +96,13 @@ class MoELayer:
             probes[0].record(stream)
         capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], inp.get("w13_scale"),
                              self.sorted_ids, self.block_expert, self.num_padded, T, k, H, I, E, self.bm, self.h,
-                             self.h_amax, stream)
+                             self.h_scale, self.ws1, stream)
         if probes:
             probes[1].record(stream)
             if addend:  # take the addend wait before the probe: the pair times the kernel alone
                 stream.wait_event(self.ev_addend)
             probes[2].record(stream)
-        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_amax, inp["w2"], inp.get("w2_scale"),
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_scale, inp["w2"], inp.get("w2_scale"),
                                         self.topk_weights, capi.MOE_DT_F32, self.sorted_ids, self.block_expert,
                                         self.num_padded, T, k, H, I, E, self.bm,
                                         self.addend if addend else None, self.ev_addend if addend else None,

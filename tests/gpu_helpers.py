@@ -26,6 +26,32 @@ def run_layer(cfg, inp_dev: dict, block_m=None, steps=1):
     return layer
 
 
+def check_routing(cfg, logits, bias, gpu_ids, gpu_w):
+    """Routing ids bit-exact against the oracle, weights to 1e-6 relative.
+
+    Grouped sigmoid routing: a token holding a score within the hazard margin
+    of an fp32 rounding midpoint (oracle.sigmoid_fp32_hazard_mask) may take the
+    other rounding of that score; such a token must then equal the oracle's
+    routing evaluated with the other rounding. Returns the tokens whose routing
+    equals the oracle's primary one (those the output is compared on)."""
+    logits = np.asarray(logits, np.float32)
+    ids, w = oracle.route(cfg.as_dict(), logits, bias)
+    same = np.all(gpu_ids == ids, axis=1)
+    if cfg.route == "grouped_sigmoid":
+        mask = oracle.sigmoid_fp32_hazard_mask(logits)
+        haz = mask.any(axis=1)
+        alt_s = np.where(mask, oracle.sigmoid_fp32_other(logits), oracle.sigmoid_fp32(logits))
+        alt_ids, alt_w = oracle.router_grouped_sigmoid_topk(logits, bias, cfg.top_k, cfg.n_group, cfg.topk_group,
+                                                            cfg.renormalize, cfg.rsf, scores=alt_s)
+        alt = haz & np.all(gpu_ids == alt_ids, axis=1)
+        assert np.all(same | alt), f"routing differs at tokens {np.nonzero(~(same | alt))[0][:10]}"
+        w = np.where(same[:, None], w, alt_w)
+    else:
+        assert np.all(same), f"routing differs at tokens {np.nonzero(~same)[0][:10]}"
+    np.testing.assert_allclose(gpu_w, w, rtol=1e-6)
+    return np.nonzero(same)[0]
+
+
 def oracle_layer(cfg, inp_cpu: dict, tokens=None):
     return oracle.moe_layer(cfg.as_dict(), synth.oracle_view(inp_cpu), tokens=tokens)
 

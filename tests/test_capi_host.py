@@ -45,8 +45,12 @@ def test_info_calls(lib):
     assert lib.moe_sorted_capacity(32, 8, 128, 16) == 32 * 8 + 128 * 15  # already a multiple of 16
     assert lib.moe_sorted_capacity(5, 3, 7, 64) == 512  # 15 + 441 = 456 -> 512
     assert lib.moe_stage2_workspace_bytes(32, 2048) == 32 * 2048 * 4 + 32 * 16 * 4
-    assert lib.moe_stage1_amax_bytes(capi.MOE_DT_FP8_E4M3, 100, 1408) == 22 * 100 * 4
-    assert lib.moe_stage1_amax_bytes(capi.MOE_DT_BF16, 100, 1408) == 0
+    # fp8 stage-1 workspace: fp32 h + per-tile amax + block counters, 256-byte aligned parts
+    rows = lib.moe_sorted_capacity(1024, 6, 64, 128)
+    up = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    want = up(rows * 1408 * 4) + up(22 * rows * 4) + up(rows // 128 * 4)
+    assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 1024, 6, 64, 1408, 128) == want
+    assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 1024, 6, 64, 1408, 128) == 0
 
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake device addresses: CPU-only check")
@@ -95,14 +99,17 @@ def test_gate_rejects(lib):
 def test_stage1_rejects(lib):
     f = lib.moe_stage1_gemm
 
-    def call(dt=0, x=P, xs=None, w=P, ws=None, s=P, be=P, npd=P, T=4, k=2, H=256, I=128, E=8, bm=16, h=P, am=None):
-        return f(dt, x, xs, w, ws, s, be, npd, T, k, H, I, E, bm, h, am, None)
+    def call(dt=0, x=P, xs=None, w=P, ws=None, s=P, be=P, npd=P, T=4, k=2, H=256, I=128, E=8, bm=16, h=P, hs=None,
+             w1=None):
+        return f(dt, x, xs, w, ws, s, be, npd, T, k, H, I, E, bm, h, hs, w1, None)
     assert call(dt=capi.MOE_DT_F32) == -2
     assert call(x=None) == -1
     assert call(bm=24) == -1
     assert call(be=None) == -1
     assert call(s=None) == -1                       # identity routing needs top_k == 1
-    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales and the amax buffer
+    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales, h_scale and the workspace
+    assert call(dt=capi.MOE_DT_FP8_E4M3, xs=P, ws=P, hs=P, w1=P, H=192) == -4  # fp8 K must be 128-aligned
+    assert call(dt=capi.MOE_DT_MXFP8_E4M3) == -2
     assert call(H=200) == -4
     assert call(I=100) == -4
     assert call(x=P + 8) == -3
@@ -112,10 +119,11 @@ def test_stage1_rejects(lib):
 def test_stage2_rejects(lib):
     f = lib.moe_stage2_gemm_accumulate
 
-    def call(dt=0, h=P, am=None, w2=P, w2s=None, wt=P, wdt=capi.MOE_DT_F32, s=P, be=P, npd=P, T=4, k=2, H=256,
+    def call(dt=0, h=P, hs=None, w2=P, w2s=None, wt=P, wdt=capi.MOE_DT_F32, s=P, be=P, npd=P, T=4, k=2, H=256,
              I=128, E=8, bm=16, add=None, ev=None, ws=P, out=P):
-        return f(dt, h, am, w2, w2s, wt, wdt, s, be, npd, T, k, H, I, E, bm, add, ev, ws, out, None)
+        return f(dt, h, hs, w2, w2s, wt, wdt, s, be, npd, T, k, H, I, E, bm, add, ev, ws, out, None)
     assert call(dt=capi.MOE_DT_FP16) == -2
+    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs h_scale and w2_scale
     assert call(out=None) == -1
     assert call(ws=None) == -1                      # top_k > 1 needs the workspace
     assert call(wdt=7) == -2

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 import oracle
+from gpu_helpers import check_routing
 from routed_shared_experts_b200 import capi, configs, synth
 
 pytestmark = pytest.mark.gpu
@@ -39,13 +40,9 @@ def test_router_grouped_config(cuda_lib, name):
     # logits and correction bias of the config's shape and distribution
     logits = torch.randn(cfg.T, cfg.E, generator=g) * 0.9
     bias = torch.randn(cfg.E, generator=g) * cfg.correction_bias_std
-    assert oracle.sigmoid_fp32_hazards(logits.numpy()) == 0
     ids, w = _route_gpu(logits, bias, cfg.top_k, capi.MOE_ROUTE_GROUPED_SIGMOID, cfg.n_group, cfg.topk_group,
                         True, cfg.rsf)
-    rid, rw = oracle.router_grouped_sigmoid_topk(logits.numpy(), bias.numpy(), cfg.top_k, cfg.n_group,
-                                                 cfg.topk_group, True, cfg.rsf)
-    assert np.array_equal(ids, rid)
-    np.testing.assert_allclose(w, rw, rtol=1e-6)
+    check_routing(cfg, logits.numpy(), bias.numpy(), ids, w)
     np.testing.assert_allclose(w.sum(1), cfg.rsf, rtol=2e-6)
 
 

@@ -174,6 +174,32 @@ def test_sigmoid_closed_forms():
     assert abs(float(s[3]) + float(s[4]) - 1.0) < 2**-23
 
 
+def test_sigmoid_other_rounding_brackets_the_double_value():
+    rng = np.random.default_rng(13)
+    l = rng.normal(0, 3, 20000).astype(np.float32)
+    v = 1.0 / (1.0 + np.exp(-l.astype(np.float64)))
+    s = mo.sigmoid_fp32(l)
+    o = oracle.sigmoid_fp32_other(l)
+    assert np.all((np.minimum(s, o) <= v) & (v <= np.maximum(s, o)))
+    # adjacent fp32 values: nothing representable strictly between them
+    s32, o32 = s.astype(np.float32), o.astype(np.float32)
+    assert np.all(np.nextafter(s32, o32) == o32)
+    # the nearest one is the primary rounding
+    assert np.all(np.abs(s - v) <= np.abs(o - v))
+    # a hazard is a value (almost) on the midpoint of the two
+    m = oracle.sigmoid_fp32_hazard_mask(l, margin_log2=-20)
+    assert np.all(np.abs(np.abs(s - v) - np.abs(o - v))[m] <= np.abs(v[m]) * 2.0**-19)
+
+
+def test_grouped_router_score_override_reproduces_default():
+    rng = np.random.default_rng(14)
+    l = rng.normal(0, 1, (50, 64)).astype(np.float32)
+    b = rng.normal(0, 0.1, 64).astype(np.float32)
+    a = oracle.router_grouped_sigmoid_topk(l, b, 6, 8, 4, True, 2.5)
+    o = oracle.router_grouped_sigmoid_topk(l, b, 6, 8, 4, True, 2.5, scores=mo.sigmoid_fp32(l))
+    assert np.array_equal(a[0], o[0]) and np.array_equal(a[1], o[1])
+
+
 def _brute_grouped(c, s, k, n_group, topk_group, rsf):
     E = len(c)
     gsize = E // n_group
