@@ -115,6 +115,28 @@ size_t moe_stage2_workspace_bytes(int T, int H);
  * counters at zero. */
 size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int I, int block_m);
 
+/* Bytes of the packed MXFP8 weight scales of one projection: which = 0 for W13
+ * ([E,2I,H] weights), which = 1 for W2 ([E,H,I] weights). 0 unless H and I are
+ * multiples of 128. */
+size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I);
+
+/* Bytes of the MXFP8 scale tiles of the stage-1 output h (capacity rows of I
+ * columns); 0 for an unsupported shape. */
+size_t moe_mx_h_scale_bytes(int T, int top_k, int E, int I, int block_m);
+
+/* moe_mx_pack_weight_scales: one-off weight preparation for MXFP8 (no
+ * counterpart on the pages; MXFP8 itself is [6106]'s BLOCK_K = 32 format).
+ * src holds the ue8m0 scale bytes row-major, [E, rows, K/32] (which = 0: W13,
+ * rows = 2I, K = H; which = 1: W2, rows = H, K = I). dst
+ * (moe_mx_weight_scale_bytes) receives them as 512-byte tiles, one per
+ * (expert, 128-row weight tile, 128-column K stage): byte (m % 32)*16 +
+ * (m / 32)*4 + b holds the scale of tile row m and K block b. For W13 the tile
+ * rows are ordered as the stage-1 kernel reads them: tile row m = rr + 16*gu +
+ * 32*qq is W13 row gu*I + (4*tile + qq)*16 + rr (16 gate rows, then their 16
+ * up rows). Checks: H % 128 == 0, I % 128 == 0. Asynchronous on `stream`. */
+moe_status_t moe_mx_pack_weight_scales(int which, const void* src, void* dst, int E, int H, int I,
+                                       moe_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 
 /* moe_router_topk: top-k routing of T tokens over E experts.
@@ -168,24 +190,32 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
  * then h_r is stored in the stage-2 operand format ([6106]: quantisation fused
  * after the activation). tcgen05 tensor cores, weights streamed by TMA, token
  * rows gathered by TMA.
- *   dtype      MOE_DT_BF16 or MOE_DT_FP8_E4M3.
- *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8) or NULL.
+ *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3 or MOE_DT_MXFP8_E4M3.
+ *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8), ue8m0 bytes
+ *              [T,H/32] row-major (MXFP8), or NULL (BF16).
  *   w13        [E,2I,H]: rows 0..I-1 gate, I..2I-1 up (K = H contiguous);
- *              w13_scale fp32 [E] (FP8) or NULL.
+ *              w13_scale fp32 [E] (FP8), the packed scale tiles of
+ *              moe_mx_pack_weight_scales(0, ...) (MXFP8), or NULL.
  *   sorted_ids / block_expert / num_padded: from moe_align_sort with the same
  *              block_m. sorted_ids == NULL selects identity routing (row r =
  *              token r, expert 0, rows padded to a multiple of block_m; used
  *              for the shared expert, E = 1, k = 1); block_expert and
  *              num_padded are then ignored.
  *   h          [capacity rows, I] (padded rows hold don't-care values):
- *              BF16: bf16. FP8: e4m3 codes, row r scaled by h_scale[r].
+ *              BF16: bf16. FP8 / MXFP8: e4m3 codes.
  *   h_scale    FP8: fp32 [capacity rows], amax(h_r)/448 (1 for an all-zero
  *              row); the codes are e4m3(h_r / h_scale[r]), round to nearest
- *              even, saturating. NULL for BF16.
+ *              even, saturating. MXFP8: moe_mx_h_scale_bytes(...) bytes of
+ *              scale tiles, one ue8m0 byte X+127 per (row, 32 columns) with
+ *              X = floor(log2 amax) - 8 (clamped to [-127,127], -127 for an
+ *              all-zero block) and codes e4m3(h * 2^-X); tile layout as in
+ *              moe_mx_pack_weight_scales with the block_m rows of one token
+ *              block per tile. NULL for BF16.
  *   ws         FP8: moe_stage1_workspace_bytes(...) bytes, zeroed once by the
  *              caller. NULL for BF16.
- * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8), I % 64 == 0, block_m in
- * {16,32,64,128,256}, 16-byte aligned x, w13, h, ws. */
+ * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8) / % 512 == 0 (MXFP8),
+ * I % 64 == 0 (% 128 for MXFP8), block_m in {16,32,64,128,256} (<= 128 for
+ * MXFP8), 16-byte aligned x, w13, h, ws and the MXFP8 scale arrays. */
 moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, const void* w13,
                              const void* w13_scale, const int32_t* sorted_ids,
                              const int32_t* block_expert, const int32_t* num_padded, int T,
@@ -202,7 +232,9 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
  * in an fp32 workspace; the epilogue that brings a token's last slot adds the
  * addend, rounds once to bf16, writes out and re-zeroes its workspace slice.
  *   dtype       as stage 1; h / h_scale are stage 1's outputs.
- *   w2          [E,H,I] (K = I contiguous); w2_scale fp32 [E] (FP8) or NULL.
+ *   w2          [E,H,I] (K = I contiguous); w2_scale fp32 [E] (FP8), the
+ *               tiles of moe_mx_pack_weight_scales(1, ...) (MXFP8; the block
+ *               scales enter the tensor-core MMA), or NULL.
  *   weights     [T*k] per slot f (routing weights, scale folded in), dtype
  *               weights_dtype = MOE_DT_F32, or MOE_DT_BF16 / MOE_DT_FP16 (the
  *               shared gate's output); NULL = 1.0.
@@ -216,8 +248,8 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
  * Identity routing (sorted_ids == NULL): as in stage 1; with top_k == 1 each
  * row's result goes straight to out (this is how the shared expert's output
  * becomes the addend of the routed call).
- * Checks: H % 128 == 0, I % 64 == 0, block_m as stage 1, 16-byte aligned h,
- * w2, out, addend, acc_ws. */
+ * Checks: H % 128 == 0, I % 64 == 0 (% 128 for MXFP8), block_m as stage 1,
+ * 16-byte aligned h, w2, out, addend, acc_ws and the MXFP8 scale arrays. */
 moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale,
                                         const void* w2, const void* w2_scale, const void* weights,
                                         int weights_dtype, const int32_t* sorted_ids,

@@ -355,8 +355,11 @@ def shared_gate(x, w, apply_sigmoid: bool = True, out_format: FloatFormat = BF16
 
 
 def silu(z):
+    """z * sigmoid(z) = z / (1 + exp(-z)); for very negative z exp(-z)
+    overflows to inf and the quotient is the correct limit, -0."""
     z = np.asarray(z, np.float64)
-    return z / (1.0 + np.exp(-z))
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
 
 
 def quantize_h(h, mode: str) -> np.ndarray:

@@ -31,6 +31,9 @@ SIGNATURES = {
     "moe_sorted_capacity": (_SZ, [_I, _I, _I, _I]),
     "moe_stage2_workspace_bytes": (_SZ, [_I, _I]),
     "moe_stage1_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "moe_mx_weight_scale_bytes": (_SZ, [_I, _I, _I, _I]),
+    "moe_mx_h_scale_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "moe_mx_pack_weight_scales": (_I, [_I, _P, _P, _I, _I, _I, _P]),
     "moe_router_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "moe_align_sort": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
@@ -106,6 +109,19 @@ def stage2_workspace_bytes(T: int, H: int) -> int:
 
 def stage1_workspace_bytes(dtype: int, T: int, top_k: int, E: int, I: int, block_m: int) -> int:
     return lib().moe_stage1_workspace_bytes(dtype, T, top_k, E, I, block_m)
+
+
+def mx_weight_scale_bytes(which: int, E: int, H: int, I: int) -> int:
+    return lib().moe_mx_weight_scale_bytes(which, E, H, I)
+
+
+def mx_h_scale_bytes(T: int, top_k: int, E: int, I: int, block_m: int) -> int:
+    return lib().moe_mx_h_scale_bytes(T, top_k, E, I, block_m)
+
+
+def moe_mx_pack_weight_scales(which, src, dst, E, H, I, stream=None):
+    _check("moe_mx_pack_weight_scales", lib().moe_mx_pack_weight_scales(
+        which, _ptr(src), _ptr(dst), E, H, I, _stream(stream)))
 
 
 def device_error(stream=None) -> int:

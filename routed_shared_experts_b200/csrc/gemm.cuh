@@ -6,12 +6,17 @@
 //   warp 0      TMA producer: weight tile (128 rows x 128 K-bytes) and token
 //               tile (BN rows x 128 K-bytes) per pipeline stage. Stage-1 token
 //               rows are gathered from x by TMA gather4 through sorted_ids.
+//               MXFP8 adds the stage's two 512-byte scale tiles.
 //   warp 1      TMEM allocator + MMA issuer (one thread): tcgen05.mma with the
 //               weights as A (M = 128) and the tokens as B (N = BN), fp32
-//               accumulator in TMEM, a ring of 2 or 4 across tiles.
-//   warps 2..  epilogue, one or two warpgroups taking alternate tiles:
+//               accumulator in TMEM, a ring of 2 or 4 across tiles. MXFP8
+//               copies the scale tiles into TMEM (tcgen05.cp) and issues the
+//               block-scaled MMA.
+//   warps 2..   epilogue, one or two warpgroups taking alternate tiles:
 //               tcgen05.ld of the accumulator, then
-//               stage 1: optional fp8 scales, SiLU(gate) * up, store h;
+//               stage 1: operand scales, SiLU(gate) * up, store h in the
+//               stage-2 operand format (bf16, e4m3 with a per-row scale, or
+//               MXFP8 with a scale per 32 columns);
 //               stage 2: scales x top-k weight, fp32 red.add into the token
 //               row, and the CTA that brings a token's last slot adds the
 //               addend, rounds once to bf16, writes out and re-zeroes.
@@ -24,7 +29,8 @@
 // output is the stage-2 addend, accumulated in the GEMM2 epilogue; commit 1:
 // the routed scale is already inside the top-k weights); ROCm/aiter PR 6106
 // "Technical Details" (per-row activation scale x per-expert weight scale on
-// the fp32 accumulator, before activation; rows follow the gather index).
+// the fp32 accumulator, before activation; rows follow the gather index;
+// MXFP8 with BLOCK_K = 32).
 #pragma once
 #include "ptx.cuh"
 
@@ -33,13 +39,18 @@ namespace moe {
 constexpr int kTileM = 128;       // weight rows per tile = MMA M
 constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte swizzle row
 constexpr int kEpiThreads = 128;  // one epilogue warpgroup
+constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
+constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)
+
+enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2 };
 
 // Epilogue warpgroups per CTA: two groups take alternate tiles (each with two
 // TMEM accumulators) so a tile's epilogue - atomics to L2 included - overlaps
-// the next tiles' main loop; 256-token tiles fill TMEM with two accumulators.
-template <int BN>
+// the next tiles' main loop. 256-token tiles fill TMEM with two accumulators,
+// and MXFP8 keeps two accumulators to leave TMEM room for the scale ring.
+template <int BN, int KIND>
 struct EpiCfg {
-  static constexpr int kGroups = BN <= 128 ? 2 : 1;
+  static constexpr int kGroups = (BN <= 128 && KIND != kMx8) ? 2 : 1;
   static constexpr int kAcc = 2 * kGroups;
   static constexpr int kThreads = 64 + kEpiThreads * kGroups;
 };
@@ -58,12 +69,14 @@ struct GemmArgs {
   float* h32;        // fp8: the unquantised h [rows, I] in fp32 (workspace)
   float* h_amax;     // fp8: per-tile row amax [n_mt][rows_cap] (workspace)
   int* blk_cnt;      // fp8: finished weight tiles per token block (workspace, self-cleaning)
-  uint8_t* hq;       // fp8: e4m3 codes of h [rows, I]
+  uint8_t* hq;       // fp8 / MXFP8: e4m3 codes of h [rows, I]
   int rows_cap;
   const float* x_scale;  // fp8: [T]
   const float* w_scale;  // fp8: [E] (stage 1: W13, stage 2: W2)
-  // stage 1 output / stage 2 input: fp8 per-row scale of h [rows]
-  float* h_scale;
+  float* h_scale;        // fp8: per-row scale of h [rows] (stage-1 output, stage-2 input)
+  // MXFP8
+  const uint8_t* wsf;  // weight scale tiles [E][n_mt][num_kb][512] (moe_mx_pack_weight_scales)
+  uint8_t* hsf;        // h scale tiles [blocks][I/128][512] (stage-1 output, stage-2 input)
   // stage 2
   const void* weights;  // [T*k] or nullptr
   int weights_dtype;    // 4 = f32, 0 = bf16, 1 = fp16
@@ -73,23 +86,35 @@ struct GemmArgs {
   __nv_bfloat16* out;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int KIND>
 struct GemmSmem {
-  static constexpr int kGroups = EpiCfg<BN>::kGroups;
-  static constexpr int kAcc = EpiCfg<BN>::kAcc;
+  static constexpr bool kMx = KIND == kMx8;
+  static constexpr int kGroups = EpiCfg<BN, KIND>::kGroups;
+  static constexpr int kAcc = EpiCfg<BN, KIND>::kAcc;
   static constexpr int kABytes = kTileM * kTileKBytes;
   static constexpr int kBBytes = BN * kTileKBytes;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOffset = STAGES * kStageBytes;
-  // full[S], empty[S], acc_full[A], acc_empty[A], drain
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
+  static constexpr int kSfBytes = kMx ? 2 * kSfTile : 0;  // A then B scale tile
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfBytes;
+  // MXFP8 stage 1: token scale bytes gathered 16 per row (4 stages) into two
+  // buffers; each gather of 4 rows (64 bytes) gets its own 128-byte-aligned slot
+  static constexpr int kStgBuf = BN / 4 * 128;
+  static constexpr int kStgBytes = kMx ? 2 * kStgBuf : 0;
+  static constexpr int kStgOffset = STAGES * kStageBytes;
+  static constexpr int kBarOffset = kStgOffset + kStgBytes;
+  // full[S], empty[S], acc_full[A], acc_empty[A], drain, staging[2]
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1 + 2;
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
   // tmem slot, abort flag, 2 pad words, producer rows[BN]; then per epilogue
   // group: ok flag + 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
   static constexpr int kGroupWords = 4 + 7 * BN;
   static constexpr int kMiscBytes = 16 + BN * 4 + kGroups * kGroupWords * 4;
   static constexpr int kBytes = kMiscOffset + kMiscBytes + 1024;  // + alignment slack
-  static constexpr int kTmemCols = (kAcc * BN < 32) ? 32 : kAcc * BN;
+  static constexpr int kAccCols = kAcc * BN;
+  static constexpr int kSfCol = kAccCols;  // first column of the scale ring
+  static constexpr int kColsNeeded = kAccCols + (kMx ? 8 * kSfSlots : 0);
+  static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 : kColsNeeded <= 128 ? 128
+                                   : kColsNeeded <= 256 ? 256 : 512;
+  static_assert(kColsNeeded <= 512, "TMEM");
 };
 
 __device__ __forceinline__ float load_weight(const void* w, int dt, int f) {
@@ -125,6 +150,16 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Shared exponent of an MXFP8 block: X = floor(log2(amax)) - 8, clamped to
+// [-127, 127]; amax = 0 gives -127 (OCP MX v1.0 conversion for e4m3 elements).
+__device__ __forceinline__ int mx_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int e;
+  frexpf(amax, &e);  // amax = m * 2^e, m in [0.5, 1): floor(log2 amax) = e - 1
+  const int x = e - 1 - 8;
+  return x < -127 ? -127 : (x > 127 ? 127 : x);
+}
+
 // Quantise the BN rows of token block `blk` from the unquantised fp32 h to
 // e4m3 with one fp32 scale per row, s = amax / 448 (amax = 0 -> s = 1), code =
 // e4m3(h / s) (round to nearest even, saturating). Run by one epilogue
@@ -155,16 +190,27 @@ __device__ __noinline__ void quantize_block_rows(const GemmArgs& g, int blk, int
   }
 }
 
-template <int BN, int STAGES, bool S1, bool FP8>
-__global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
-    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
-  using L = GemmSmem<BN, STAGES>;
+// Byte offset of the scale of (row n, K block kb of the 4 in a stage) inside
+// a 512-byte MXFP8 scale tile: 32 row positions x 16 bytes, each holding the
+// 4 row groups (n / 32) x 4 K blocks. tcgen05.cp.32x128b.warpx4 moves the tile
+// so that TMEM lane n % 32 (and its copies in the other lane quarters) holds,
+// in column n / 32, the four K-block bytes of row n.
+__host__ __device__ constexpr int sf_tile_offset(int n, int kb) { return (n % 32) * 16 + (n / 32) * 4 + kb; }
+
+template <int BN, int STAGES, bool S1, int KIND>
+__global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmS, const GemmArgs g) {
+  using L = GemmSmem<BN, STAGES, KIND>;
+  constexpr bool FP8 = KIND == kFp8;
+  constexpr bool MX = KIND == kMx8;
   constexpr int G = L::kGroups;
   constexpr int NACC = L::kAcc;
-  constexpr int KE = FP8 ? 128 : 64;  // K elements per stage
-  constexpr int kUmmaKBytes = 32;     // K bytes per MMA: 16 bf16 or 32 e4m3
+  constexpr int KE = KIND == kBf16 ? 64 : 128;  // K elements per stage
+  constexpr int kUmmaKBytes = 32;               // K bytes per MMA: 16 bf16 or 32 e4m3
   constexpr uint32_t kIdesc = FP8 ? idesc_e4m3(kTileM, BN) : idesc_bf16(kTileM, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
+  static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
 
   extern __shared__ uint8_t smem_raw[];
@@ -174,6 +220,8 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* drain = acc_empty + NACC;
+  uint64_t* stg_full = drain + 1;  // MXFP8 stage 1: token-scale staging buffers
+  uint8_t* stg = smem + L::kStgOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* rows_sm = reinterpret_cast<int*>(tmem_slot + 4);
@@ -192,6 +240,8 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
       mbar_init(&acc_empty[a], kEpiThreads);
     }
     mbar_init(drain, 1);
+    mbar_init(&stg_full[0], 1);
+    mbar_init(&stg_full[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -216,7 +266,21 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t pending = 0, pend_parity = 0;  // stages armed and not yet re-acquired
+    uint32_t stg_phase = 0;                 // MXFP8 stage 1: parity bits of the two staging buffers
+    uint32_t stg_pending = 0;
     bool ok = true;
+    // MXFP8 stage 1: gather the token rows' scale bytes of stages [4c, 4c+4)
+    // (16 bytes per row) into staging buffer c % 2.
+    auto issue_stage_scales = [&](int c) {
+      const int b = c & 1;
+      fence_proxy_async_smem();  // earlier generic reads of this buffer come first
+      mbar_arrive_expect_tx(&stg_full[b], BN * 16);
+#pragma unroll 4
+      for (int q = 0; q < BN / 4; ++q)
+        tma_gather4(stg + b * L::kStgBuf + q * 128, &tmS, &stg_full[b], c * 16, rows_sm[4 * q],
+                    rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
+      stg_pending |= 1u << b;
+    };
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const int blk = tile / g.n_mt;
       const int mt = tile - blk * g.n_mt;
@@ -235,31 +299,63 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
           rows_sm[i] = row;
         }
         __syncwarp();
+        if (MX && lane == 0) issue_stage_scales(0);
       }
       for (int kb = 0; kb < g.num_kb; ++kb) {
+        uint8_t* a_dst = smem + stage * L::kStageBytes;
+        uint8_t* b_dst = a_dst + L::kABytes;
+        uint8_t* sfa_dst = b_dst + L::kBBytes;
+        uint8_t* sfb_dst = sfa_dst + kSfTile;
         if (lane == 0) {
           ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
-          if (ok) {
-            pending &= ~(1u << stage);
-            uint8_t* a_dst = smem + stage * L::kStageBytes;
-            uint8_t* b_dst = a_dst + L::kABytes;
-            mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
-            if (S1) {
-              tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
-#pragma unroll 4
-              for (int q = 0; q < BN / 4; ++q)
-                tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
-                            rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
-            } else {
-              tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
-              tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+          if (ok && MX && S1 && (kb & 3) == 0) {
+            const int c = kb >> 2, b = c & 1;
+            ok = mbar_wait(&stg_full[b], (stg_phase >> b) & 1u, abort_flag);
+            if (ok) {
+              stg_phase ^= 1u << b;
+              stg_pending &= ~(1u << b);
+              if ((c + 1) * 4 < g.num_kb) issue_stage_scales(c + 1);
             }
-            pending |= 1u << stage;
-            pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        if (MX && S1) {
+          // this stage's 4 K-block bytes of every token row, into the tile layout
+          // (row n sits at byte (n / 4) * 128 + (n % 4) * 16 of its staging buffer)
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(stg + ((kb >> 2) & 1) * L::kStgBuf);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(sfb_dst);
+          for (int n = lane; n < BN; n += 32)
+            dst[sf_tile_offset(n, 0) / 4] = src[(n / 4) * 32 + (n % 4) * 4 + (kb & 3)];
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          pending &= ~(1u << stage);
+          uint32_t bytes = L::kABytes + L::kBBytes;
+          if (MX) bytes += S1 ? kSfTile : 2 * kSfTile;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          if (S1) {
+            tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+#pragma unroll 4
+            for (int q = 0; q < BN / 4; ++q)
+              tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
+                          rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
+          } else {
+            tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+          }
+          if (MX) {
+            const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
+            bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
+            if (!S1)
+              bulk_load(sfb_dst, g.hsf + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile, kSfTile,
+                        &full[stage], pol_x);
+          }
+          pending |= 1u << stage;
+          pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+        }
+        __syncwarp();
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -270,12 +366,15 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
     if (!ok && lane == 0) {
       for (int s = 0; s < STAGES; ++s)
         if ((pending >> s) & 1u) drain_wait(&full[s], (pend_parity >> s) & 1u);
+      for (int b = 0; b < 2; ++b)
+        if ((stg_pending >> b) & 1u) drain_wait(&stg_full[b], (stg_phase >> b) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    uint32_t sf_slot = 0;
     int j = 0;  // local tile counter: accumulator j % NACC, use (j / NACC)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
       const int acc = j % NACC;
@@ -294,17 +393,32 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
           const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
           const uint64_t adesc = sw128_kmajor_desc(a_addr);
           const uint64_t bdesc = sw128_kmajor_desc(a_addr + L::kABytes);
+          uint32_t tsfa = 0, tsfb = 0;
+          if (MX) {
+            // scale tiles of this stage -> TMEM ring slot (A: 4 columns, B: the next 4)
+            tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol) + sf_slot * 8;
+            tsfb = tsfa + 4;
+            const uint32_t sf_addr = a_addr + L::kABytes + L::kBBytes;
+            tmem_cp_32x128b_x4(tsfa, plain_rows16_desc(sf_addr));
+            tmem_cp_32x128b_x4(tsfb, plain_rows16_desc(sf_addr + kSfTile));
+            sf_slot = (sf_slot + 1) % kSfSlots;
+          }
 #pragma unroll
           for (int kk = 0; kk < kTileKBytes / kUmmaKBytes; ++kk) {
             // +32 bytes along K inside the swizzle row: +2 in the (addr >> 4) field
             const uint64_t adv = static_cast<uint64_t>(kk * (kUmmaKBytes >> 4));
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if (FP8)
+            if (MX) {
+              // K block kk of the stage: byte kk of each scale column
+              const uint32_t sel = static_cast<uint32_t>(kk) << 30;
+              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, BN, kk), tsfa | sel, tsfb | sel, accum);
+            } else if (FP8) {
               umma_f8(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
-            else
+            } else {
               umma_f16(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
+            }
           }
-          umma_commit(&empty[stage]);  // smem stage free once these MMAs finish
+          umma_commit(&empty[stage]);  // smem stage free once these MMAs (and copies) finish
         }
         __syncwarp();
         if (++stage == STAGES) {
@@ -368,9 +482,11 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
 
       if (S1) {
         // Lanes 0..15 of quarter q hold gate features 16q..16q+15 of this
-        // 64-feature tile, lanes 16..31 the matching up features.
+        // 64-feature tile, lanes 16..31 the matching up features. Lanes 0..15
+        // finish the even columns, lanes 16..31 the odd ones.
         const int feat = mt * 64 + 16 * q + (lane & 15);
         const bool lo = lane < 16;
+        float hv_keep[MX ? BN / 2 : 1];  // MXFP8: h of this thread's columns until the block scale is known
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           float v[16];
@@ -394,12 +510,13 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
               up *= sc;
             }
             const float hv = gt / (1.0f + expf(-gt)) * up;
-            if (feat < g.I) {
+            if (!MX && feat < g.I) {
               if (FP8) g.h32[static_cast<size_t>(r) * g.I + feat] = hv;
               else g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
             }
-            if (FP8) {
-              // per-row amax of this tile's 16 features of the half-warp
+            if (MX) hv_keep[(c0 + i) / 2] = hv;
+            if (FP8 || MX) {
+              // amax over this half-warp's 16 features of column c
               float m = fabsf(hv);
               m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
               m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
@@ -407,6 +524,26 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
               m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
               if ((lane & 15) == 0) amax_part[q * BN + c] = m;
             }
+          }
+        }
+        if (MX) {
+          // One MX block = 32 features = lane quarters 2p and 2p+1 of the tile
+          // (ROCm/aiter PR 6106: BLOCK_K = 32): shared exponent from the pair's
+          // amax, codes e4m3(h * 2^-X), one ue8m0 byte X + 127 per (row, block),
+          // written into stage 2's scale tile layout.
+          named_bar_sync(bar_id, kEpiThreads);
+          const int kblk = feat / 32;  // K block of stage 2
+          const size_t tile_base = (static_cast<size_t>(blk) * (g.I / 128) + kblk / 4) * kSfTile;
+#pragma unroll
+          for (int i = 0; i < BN / 2; ++i) {
+            const int c = 2 * i + (lo ? 0 : 1);
+            const float amax = fmaxf(amax_part[q * BN + c], amax_part[(q ^ 1) * BN + c]);
+            const int X = mx_exponent(amax);
+            const float v = ldexpf(hv_keep[i], -X);
+            const uint8_t code = static_cast<uint8_t>(cvt_e4m3x2(v, 0.f) & 0xFF);
+            if (feat < g.I) g.hq[static_cast<size_t>(blk * BN + c) * g.I + feat] = code;
+            if ((q & 1) == 0 && (lane & 15) == 0)
+              g.hsf[tile_base + sf_tile_offset(c, kblk & 3)] = static_cast<uint8_t>(X + 127);
           }
         }
         if (FP8) {
@@ -498,6 +635,39 @@ __global__ void __launch_bounds__(EpiCfg<BN>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// Weight scale tiles for MXFP8 (one-off weight preparation). src is the
+// row-major [E][rows][K/32] ue8m0 bytes; dst gets, per (expert, weight tile,
+// stage), the 512-byte tile of the 128 A-operand rows x 4 K blocks in
+// sf_tile_offset order. W13 tiles follow the stage-1 A layout, whose row m
+// (m = rr + 16*gu + 32*qq) is W13 row gu*I + (4*mt + qq)*16 + rr; W2 tiles are
+// 128 consecutive rows.
+__global__ void k_mx_pack_weight_scales(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int E, int rows,
+                                        int K, int I, int w13) {
+  const int kbs = K / 32;    // K blocks per row
+  const int n_kg = K / 128;  // stages per tile
+  const int n_mt = w13 ? I / 64 : rows / 128;
+  const size_t n_out = static_cast<size_t>(E) * n_mt * n_kg * kSfTile;
+  for (size_t o = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; o < n_out;
+       o += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int within = static_cast<int>(o % kSfTile);
+    size_t t = o / kSfTile;
+    const int kg = static_cast<int>(t % n_kg);
+    t /= n_kg;
+    const int mt = static_cast<int>(t % n_mt);
+    const int e = static_cast<int>(t / n_mt);
+    const int m0 = within / 16, m1 = (within % 16) / 4, kb = within % 4;
+    const int m = m0 + 32 * m1;  // A-operand row of the tile
+    int row;
+    if (w13) {
+      const int rr = m % 16, gu = (m / 16) % 2, qq = m / 32;
+      row = gu * I + (4 * mt + qq) * 16 + rr;
+    } else {
+      row = mt * 128 + m;
+    }
+    dst[o] = src[(static_cast<size_t>(e) * rows + row) * kbs + kg * 4 + kb];
   }
 }
 

@@ -72,7 +72,8 @@ EncodeTiledFn encode_fn() {
 // Tiled map with the 128-byte swizzle; dims/box innermost first, strides in
 // bytes for dims 1..rank-1.
 moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
-                      const cuuint64_t* strides, const cuuint32_t* box) {
+                      const cuuint64_t* strides, const cuuint32_t* box,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn f = encode_fn();
   if (!f) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
@@ -80,7 +81,7 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
   }
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   const CUresult r = f(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, es,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (CUresult %d)",
@@ -92,18 +93,19 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
 
 // ------------------------------------------------------------ GEMM dispatch
 
-template <int BN>
+template <int BN, int KIND>
 constexpr int stages_for() {
-  // ~192 KB of pipeline per CTA, one CTA per SM
+  // ~190 KB of pipeline per CTA, one CTA per SM
+  if (KIND == moe::kMx8) return BN == 16 ? 10 : BN == 32 ? 9 : BN == 64 ? 7 : 5;
   return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : BN == 128 ? 6 : 4;
 }
 
-template <int BN, bool S1, bool FP8>
-moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
-                            cudaStream_t s) {
-  constexpr int ST = stages_for<BN>();
-  using L = moe::GemmSmem<BN, ST>;
-  auto kern = moe::k_moe_gemm<BN, ST, S1, FP8>;
+template <int BN, bool S1, int KIND>
+moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
+                            const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
+  constexpr int ST = stages_for<BN, KIND>();
+  using L = moe::GemmSmem<BN, ST, KIND>;
+  auto kern = moe::k_moe_gemm<BN, ST, S1, KIND>;
   static std::atomic<int> attr_set[64];
   int dev = 0;
   MOE_CK(cudaGetDevice(&dev));
@@ -113,22 +115,32 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
   }
   int grid = max_tiles < num_sms() ? max_tiles : num_sms();
   if (grid < 1) grid = 1;
-  kern<<<grid, moe::EpiCfg<BN>::kThreads, L::kBytes, s>>>(ta, tb, g);
+  kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, ts, g);
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
 
-template <bool S1, bool FP8>
-moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g,
-                         int max_tiles, cudaStream_t s) {
+template <bool S1, int KIND>
+moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
+                         const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   switch (bm) {
-    case 16: return launch_gemm_bn<16, S1, FP8>(ta, tb, g, max_tiles, s);
-    case 32: return launch_gemm_bn<32, S1, FP8>(ta, tb, g, max_tiles, s);
-    case 64: return launch_gemm_bn<64, S1, FP8>(ta, tb, g, max_tiles, s);
-    case 128: return launch_gemm_bn<128, S1, FP8>(ta, tb, g, max_tiles, s);
-    case 256: return launch_gemm_bn<256, S1, FP8>(ta, tb, g, max_tiles, s);
+    case 16: return launch_gemm_bn<16, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+    case 32: return launch_gemm_bn<32, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+    case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+    case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+    case 256:
+      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+      break;
   }
   return MOE_ERR_INVALID_ARG;
+}
+
+template <bool S1>
+moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
+                              const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
+  if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, ts, g, max_tiles, s);
+  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, ts, g, max_tiles, s);
+  return launch_gemm<S1, moe::kBf16>(bm, ta, tb, ts, g, max_tiles, s);
 }
 
 // Padded sorted length bound T*k + E*(bm-1), rounded up to whole blocks.
@@ -302,26 +314,33 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
                              int top_k, int H, int I, int E, int block_m, void* h, void* h_scale, void* ws,
                              moe_stream_t stream) {
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
-  if (dtype != MOE_DT_BF16 && !fp8) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const bool mx = dtype == MOE_DT_MXFP8_E4M3;
+  if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!x || !w13 || !h) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
   if (fp8 && (!x_scale || !w13_scale || !h_scale || !ws)) return MOE_ERR_INVALID_ARG;
-  if (H % (fp8 ? 128 : 64) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(w13) || !aligned16(h) || (ws && !aligned16(ws))) return MOE_ERR_ALIGNMENT;
+  if (mx && (!x_scale || !w13_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+  if (mx && block_m > 128) return MOE_ERR_INVALID_ARG;
+  if (H % (dtype == MOE_DT_BF16 ? 64 : 128) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (mx && (H % 512 != 0 || I % 128 != 0)) return MOE_ERR_ALIGNMENT;  // whole 16-byte scale runs, 4-block tiles
+  if (!aligned16(x) || !aligned16(w13) || !aligned16(h) || (ws && !aligned16(ws)) ||
+      (mx && (!aligned16(x_scale) || !aligned16(w13_scale) || !aligned16(h_scale))))
+    return MOE_ERR_ALIGNMENT;
 
-  const int es = fp8 ? 1 : 2;
-  const int ke = fp8 ? 128 : 64;
+  const bool b16 = dtype == MOE_DT_BF16;
+  const int es = b16 ? 2 : 1;
+  const int ke = b16 ? 64 : 128;
   const size_t rows_cap = capacity(T, top_k, E, block_m);  // identity routing: T rounded up to block_m
   const int cap_blocks = static_cast<int>(rows_cap / block_m);
-  const CUtensorMapDataType tdt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
 
   // W13 as 5-D (K, row-in-16, gate|up, 16-row group, expert): one box brings
   // 16 gate rows then the 16 matching up rows for four consecutive groups, so
   // the 128 weight rows of a tile pair gate and up inside each 32-lane quarter.
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ts;
   {
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(H), 16, 2, static_cast<cuuint64_t>(I / 16),
                                 static_cast<cuuint64_t>(E)};
@@ -336,6 +355,16 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), 1};
     moe_status_t r = make_map(&tb, tdt, 2, x, dims, st, box);
+    if (r != MOE_OK) return r;
+  }
+  ts = tb;
+  if (mx) {
+    // token scale bytes [T][H/32], gathered 16 bytes (4 stages) per row
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H / 32), static_cast<cuuint64_t>(T)};
+    const cuuint64_t st[1] = {static_cast<cuuint64_t>(H / 32)};
+    const cuuint32_t box[2] = {16, 1};
+    moe_status_t r = make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, x_scale, dims, st, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
     if (r != MOE_OK) return r;
   }
   moe::GemmArgs g{};
@@ -361,13 +390,15 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     g.h_scale = static_cast<float*>(h_scale);
     g.x_scale = static_cast<const float*>(x_scale);
     g.w_scale = static_cast<const float*>(w13_scale);
+  } else if (mx) {
+    g.hq = static_cast<uint8_t*>(h);
+    g.hsf = static_cast<uint8_t*>(h_scale);
+    g.wsf = static_cast<const uint8_t*>(w13_scale);
   } else {
     g.h = static_cast<__nv_bfloat16*>(h);
   }
   const int max_tiles = cap_blocks * g.n_mt;
-  cudaStream_t s = as_stream(stream);
-  return fp8 ? launch_gemm<true, true>(block_m, ta, tb, g, max_tiles, s)
-             : launch_gemm<true, false>(block_m, ta, tb, g, max_tiles, s);
+  return launch_gemm_kind<true>(dtype, block_m, ta, tb, ts, g, max_tiles, as_stream(stream));
 }
 
 moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale, const void* w2,
@@ -377,26 +408,30 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
                                         int block_m, const void* addend, moe_event_t addend_ready, void* acc_ws,
                                         void* out, moe_stream_t stream) {
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
-  if (dtype != MOE_DT_BF16 && !fp8) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const bool mx = dtype == MOE_DT_MXFP8_E4M3;
+  if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
   if (top_k > 1 && !acc_ws) return MOE_ERR_INVALID_ARG;
-  if (fp8 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if ((fp8 || mx) && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (mx && block_m > 128) return MOE_ERR_INVALID_ARG;
   if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
     return MOE_ERR_UNSUPPORTED_DTYPE;
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;
   if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)) ||
-      (acc_ws && !aligned16(acc_ws)))
+      (acc_ws && !aligned16(acc_ws)) || (mx && (!aligned16(h_scale) || !aligned16(w2_scale))))
     return MOE_ERR_ALIGNMENT;
 
-  const int es = fp8 ? 1 : 2;
-  const int ke = fp8 ? 128 : 64;
+  const bool b16 = dtype == MOE_DT_BF16;
+  const int es = b16 ? 2 : 1;
+  const int ke = b16 ? 64 : 128;
   const size_t rows_cap = capacity(T, top_k, E, block_m);
   const int cap_blocks = static_cast<int>(rows_cap / block_m);
-  const CUtensorMapDataType tdt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUtensorMap ta, tb;
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
@@ -431,15 +466,45 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.rows_cap = static_cast<int>(rows_cap);
   g.weights = weights;
   g.weights_dtype = weights_dtype;
-  g.h_scale = fp8 ? const_cast<float*>(static_cast<const float*>(h_scale)) : nullptr;
-  g.w_scale = fp8 ? static_cast<const float*>(w2_scale) : nullptr;
+  if (fp8) {
+    g.h_scale = const_cast<float*>(static_cast<const float*>(h_scale));
+    g.w_scale = static_cast<const float*>(w2_scale);
+  } else if (mx) {
+    g.hsf = const_cast<uint8_t*>(static_cast<const uint8_t*>(h_scale));
+    g.wsf = static_cast<const uint8_t*>(w2_scale);
+  }
   g.addend = static_cast<const __nv_bfloat16*>(addend);
   g.ws = static_cast<float*>(acc_ws);
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
-  return fp8 ? launch_gemm<false, true>(block_m, ta, tb, g, max_tiles, s)
-             : launch_gemm<false, false>(block_m, ta, tb, g, max_tiles, s);
+  return launch_gemm_kind<false>(dtype, block_m, ta, tb, tb, g, max_tiles, s);
+}
+
+size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I) {
+  if (E < 1 || H < 1 || I < 1 || H % 128 != 0 || I % 128 != 0) return 0;
+  const size_t tiles = which == 0 ? static_cast<size_t>(I / 64) * (H / 128) : static_cast<size_t>(H / 128) * (I / 128);
+  return static_cast<size_t>(E) * tiles * moe::kSfTile;
+}
+
+size_t moe_mx_h_scale_bytes(int T, int top_k, int E, int I, int block_m) {
+  if (T < 1 || top_k < 1 || E < 1 || I < 1 || I % 128 != 0 || !valid_block_m(block_m) || block_m > 128) return 0;
+  return capacity(T, top_k, E, block_m) / block_m * (I / 128) * moe::kSfTile;
+}
+
+moe_status_t moe_mx_pack_weight_scales(int which, const void* src, void* dst, int E, int H, int I,
+                                       moe_stream_t stream) {
+  if (!src || !dst || (which != 0 && which != 1)) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || H < 1 || I < 1) return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || I % 128 != 0) return MOE_ERR_SHAPE;
+  const int rows = which == 0 ? 2 * I : H;
+  const int K = which == 0 ? H : I;
+  const size_t n = moe_mx_weight_scale_bytes(which, E, H, I);
+  const int blocks = static_cast<int>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  moe::k_mx_pack_weight_scales<<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), E, rows, K, I, which == 0 ? 1 : 0);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
 }
 
 moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, const void* h_scale, const void* w2,
@@ -450,13 +515,15 @@ moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, cons
                                                   void* out, moe_stream_t stream) {
   // The argument checks of moe_stage2_gemm_accumulate, repeated here so that
   // nothing (not even the clearing memset) is enqueued for an invalid call.
-  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && dtype != MOE_DT_MXFP8_E4M3)
+    return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  if (dtype == MOE_DT_FP8_E4M3 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DT_BF16 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_DT_MXFP8_E4M3 && (block_m > 128 || I % 128 != 0)) return MOE_ERR_INVALID_ARG;
   if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
     return MOE_ERR_UNSUPPORTED_DTYPE;
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;

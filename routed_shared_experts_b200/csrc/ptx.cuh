@@ -187,6 +187,43 @@ __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// Block-scaled MMA, e4m3 operands with one ue8m0 scale per 32 K elements of
+// every row of A and B. tsfa / tsfb: TMEM addresses of the scale tiles; bits
+// [30,32) of each carry the byte (K block) the MMA reads, mirrored in the
+// descriptor's scale-factor id fields (see idesc_mx).
+__device__ __forceinline__ void umma_mx8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Shared memory -> TMEM: 32 rows x 16 bytes, written to TMEM lanes 0..31 of
+// the destination columns and repeated into the other three lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// Plain bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory accesses with later
+// async-proxy (TMA, tcgen05) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Arrives once on `bar` when all tcgen05 operations issued so far by this
 // thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -223,6 +260,26 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
   return d;
+}
+
+// Shared-memory descriptor of a no-swizzle K-major operand whose 16-byte rows
+// are contiguous: 8-row core matrices 128 bytes apart (stride byte offset),
+// version 1, layout SWIZZLE_NONE. Used as the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t plain_rows16_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: B scale id [4,6),
+// A/B format e4m3 (0) at [7,10)/[10,13), K-major, N >> 3 at [17,23), scale
+// format ue8m0 (1) at bit 23, M >> 4 at [24,29), A scale id [29,31).
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
 }
 
 // Instruction descriptor (kind::f16 / kind::f8f6f4): D fp32 [4,6) = 1,

@@ -52,8 +52,23 @@ class MoELayer:
         self.h = torch.empty((cap, I), dtype=hdt, device=dev)
         self.h_s = torch.empty((cap_s, Is), dtype=hdt, device=dev)
         fp8 = cfg.dtype == "fp8"
-        self.h_scale = torch.empty(cap, dtype=torch.float32, device=dev) if fp8 else None
-        self.h_scale_s = torch.empty(cap_s, dtype=torch.float32, device=dev) if fp8 else None
+        mx = cfg.dtype == "mxfp8"
+        self.h_scale = self.h_scale_s = None
+        if fp8:
+            self.h_scale = torch.empty(cap, dtype=torch.float32, device=dev)
+            self.h_scale_s = torch.empty(cap_s, dtype=torch.float32, device=dev)
+        elif mx:
+            self.h_scale = torch.zeros(capi.mx_h_scale_bytes(T, k, E, I, bm), dtype=torch.uint8, device=dev)
+            self.h_scale_s = torch.zeros(capi.mx_h_scale_bytes(T, 1, 1, Is, bm), dtype=torch.uint8, device=dev)
+        # MXFP8 weight scales in the kernels' tile layout (one-off preparation)
+        self.wsc = {}
+        for name, which, e, inter in (("w13", 0, E, I), ("w2", 1, E, I), ("w13s", 0, 1, Is), ("w2s", 1, 1, Is)):
+            if mx:
+                dst = torch.empty(capi.mx_weight_scale_bytes(which, e, H, inter), dtype=torch.uint8, device=dev)
+                capi.moe_mx_pack_weight_scales(which, inp[name + "_scale"].contiguous(), dst, e, H, inter)
+                self.wsc[name] = dst
+            else:
+                self.wsc[name] = inp.get(name + "_scale")
         ws1 = capi.stage1_workspace_bytes(self.dt, T, k, E, I, bm)
         ws1s = capi.stage1_workspace_bytes(self.dt, T, 1, 1, Is, bm)
         self.ws1 = torch.zeros(ws1, dtype=torch.uint8, device=dev) if ws1 else None  # zeroed once
@@ -75,10 +90,10 @@ class MoELayer:
         T, H, Is = cfg.T, cfg.H, cfg.Is
         if self.gate is not None:
             capi.shared_expert_gate_dot(capi.MOE_DT_BF16, inp["x"], inp["w_gate"], True, self.gate, stream)
-        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13s"], inp.get("w13s_scale"),
+        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13s"], self.wsc["w13s"],
                              None, None, None, T, 1, H, Is, 1, self.bm, self.h_s, self.h_scale_s, self.ws1_s, stream)
         wdt = capi.MOE_DT_BF16 if self.gate is not None else capi.MOE_DT_F32
-        capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_scale_s, inp["w2s"], inp.get("w2s_scale"),
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_scale_s, inp["w2s"], self.wsc["w2s"],
                                         self.gate, wdt, None, None, None, T, 1, H, Is, 1, self.bm, None, None,
                                         None, self.addend, stream)
 
@@ -94,7 +109,7 @@ class MoELayer:
                             self.expert_offsets, self.num_padded, stream)
         if probes:
             probes[0].record(stream)
-        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], inp.get("w13_scale"),
+        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], self.wsc["w13"],
                              self.sorted_ids, self.block_expert, self.num_padded, T, k, H, I, E, self.bm, self.h,
                              self.h_scale, self.ws1, stream)
         if probes:
@@ -102,7 +117,7 @@ class MoELayer:
             if addend:  # take the addend wait before the probe: the pair times the kernel alone
                 stream.wait_event(self.ev_addend)
             probes[2].record(stream)
-        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_scale, inp["w2"], inp.get("w2_scale"),
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_scale, inp["w2"], self.wsc["w2"],
                                         self.topk_weights, capi.MOE_DT_F32, self.sorted_ids, self.block_expert,
                                         self.num_padded, T, k, H, I, E, self.bm,
                                         self.addend if addend else None, self.ev_addend if addend else None,

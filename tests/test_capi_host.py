@@ -51,6 +51,11 @@ def test_info_calls(lib):
     want = up(rows * 1408 * 4) + up(22 * rows * 4) + up(rows // 128 * 4)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 1024, 6, 64, 1408, 128) == want
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 1024, 6, 64, 1408, 128) == 0
+    # MXFP8 scale tiles: 512 bytes per (expert, 128-row tile, 128-column stage)
+    assert lib.moe_mx_weight_scale_bytes(0, 256, 7168, 2048) == 256 * (2048 // 64) * (7168 // 128) * 512
+    assert lib.moe_mx_weight_scale_bytes(1, 256, 7168, 2048) == 256 * (7168 // 128) * (2048 // 128) * 512
+    assert lib.moe_mx_h_scale_bytes(4096, 8, 256, 2048, 128) == \
+        lib.moe_sorted_capacity(4096, 8, 256, 128) // 128 * 16 * 512
 
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake device addresses: CPU-only check")
@@ -109,7 +114,9 @@ def test_stage1_rejects(lib):
     assert call(s=None) == -1                       # identity routing needs top_k == 1
     assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales, h_scale and the workspace
     assert call(dt=capi.MOE_DT_FP8_E4M3, xs=P, ws=P, hs=P, w1=P, H=192) == -4  # fp8 K must be 128-aligned
-    assert call(dt=capi.MOE_DT_MXFP8_E4M3) == -2
+    assert call(dt=capi.MOE_DT_MXFP8_E4M3) == -1      # MXFP8 needs its scale arrays
+    assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, H=384, I=128) == -3  # H % 512 for the token scales
+    assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, H=512, I=128, bm=256) == -1
     assert call(H=200) == -4
     assert call(I=100) == -4
     assert call(x=P + 8) == -3

@@ -26,7 +26,7 @@ MULTI = configs.small(configs.DECODE_BF16, name="multi_bf16", T=53, H=384, E=16,
 def _static_stage2(layer, out):
     cfg, inp = layer.cfg, layer.inp
     capi.moe_stage2_gemm_accumulate_static_ws(
-        layer.dt, layer.h, layer.h_scale, inp["w2"], inp.get("w2_scale"), layer.topk_weights, capi.MOE_DT_F32,
+        layer.dt, layer.h, layer.h_scale, inp["w2"], layer.wsc["w2"], layer.topk_weights, capi.MOE_DT_F32,
         layer.sorted_ids, layer.block_expert, layer.num_padded, cfg.T, cfg.top_k, cfg.H, cfg.I, cfg.E, layer.bm,
         layer.addend, None, out)
 
