@@ -95,9 +95,9 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
 
 template <int BN, int KIND>
 constexpr int stages_for() {
-  // ~190 KB of pipeline per CTA, one CTA per SM
+  // as many stages as fit in 227 KB of shared memory, one CTA per SM
   if (KIND == moe::kMx8) return BN == 16 ? 10 : BN == 32 ? 9 : BN == 64 ? 7 : 5;
-  return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : BN == 128 ? 6 : 4;
+  return BN == 16 ? 12 : BN == 32 ? 11 : BN == 64 ? 8 : BN == 128 ? 6 : 4;
 }
 
 template <int BN, bool S1, int KIND>
