@@ -334,7 +334,8 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   const int es = b16 ? 2 : 1;
   const int ke = b16 ? 64 : 128;
   const size_t rows_cap = capacity(T, top_k, E, block_m);  // identity routing: T rounded up to block_m
-  const int cap_blocks = static_cast<int>(rows_cap / block_m);
+  // identity routing launches over the blocks that hold tokens only
+  const int cap_blocks = sorted_ids ? static_cast<int>(rows_cap / block_m) : (T + block_m - 1) / block_m;
   const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
 
   // W13 as 5-D (K, row-in-16, gate|up, 16-row group, expert): one box brings
@@ -371,7 +372,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   g.sorted_ids = sorted_ids;
   g.block_expert = block_expert;
   g.num_padded = num_padded;
-  g.identity_rows = static_cast<int>(rows_cap);
+  g.identity_rows = cap_blocks * block_m;
   g.cap_blocks = cap_blocks;
   g.T = T;
   g.top_k = top_k;
@@ -430,7 +431,8 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   const int es = b16 ? 2 : 1;
   const int ke = b16 ? 64 : 128;
   const size_t rows_cap = capacity(T, top_k, E, block_m);
-  const int cap_blocks = static_cast<int>(rows_cap / block_m);
+  // identity routing launches over the blocks that hold tokens only
+  const int cap_blocks = sorted_ids ? static_cast<int>(rows_cap / block_m) : (T + block_m - 1) / block_m;
   const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUtensorMap ta, tb;
   {
@@ -455,7 +457,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.sorted_ids = sorted_ids;
   g.block_expert = block_expert;
   g.num_padded = num_padded;
-  g.identity_rows = static_cast<int>(rows_cap);
+  g.identity_rows = cap_blocks * block_m;
   g.cap_blocks = cap_blocks;
   g.T = T;
   g.top_k = top_k;
