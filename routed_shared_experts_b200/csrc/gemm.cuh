@@ -160,33 +160,83 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   return x < -127 ? -127 : (x > 127 ? 127 : x);
 }
 
-// Quantise the BN rows of token block `blk` from the unquantised fp32 h to
-// e4m3 with one fp32 scale per row, s = amax / 448 (amax = 0 -> s = 1), code =
-// e4m3(h / s) (round to nearest even, saturating). Run by one epilogue
-// warpgroup (128 threads, named barrier `bar_id`) after it has acquired every
-// weight tile of the block; `scale_sm` is BN floats of its shared memory.
+// Quantise the rows of token block `blk` that hold a slot from the
+// unquantised fp32 h to e4m3 with one fp32 scale per row, s = amax / 448
+// (amax = 0 -> s = 1), code = e4m3(h * (1 / s)) (round to nearest even,
+// saturating; the fp32 reciprocal is taken once per row). Padding rows are
+// left as they are: stage 2 skips their output columns, and each column of
+// the MMA depends on its own row of h only. Run by one epilogue warpgroup
+// (128 threads, named barrier `bar_id`) after it has acquired every weight
+// tile of the block. `tok_sm` holds the token of each of the BN columns (-1 =
+// padding); `rows_sm` (BN ints) and `inv_sm` (BN + 1 words) are its shared scratch.
+// The pass reads the rows' fp32 values from L2, so every thread keeps
+// kQuantUnroll chunks of loads in flight before converting any of them.
+constexpr int kQuantUnroll = 8;
 template <int BN>
-__device__ __noinline__ void quantize_block_rows(const GemmArgs& g, int blk, int et, int bar_id, float* scale_sm) {
-  for (int c = et; c < BN; c += kEpiThreads) {
-    const int r = blk * BN + c;
-    float m = 0.f;
-    for (int t = 0; t < g.n_mt; ++t) m = fmaxf(m, __ldcg(g.h_amax + static_cast<size_t>(t) * g.rows_cap + r));
-    const float sc = m > 0.f ? m / 448.0f : 1.0f;
-    scale_sm[c] = sc;
-    g.h_scale[r] = sc;
+__device__ __noinline__ void quantize_block_rows(const GemmArgs& g, int blk, int et, int bar_id, const int* tok_sm,
+                                                 int* rows_sm, float* inv_sm) {
+  named_bar_sync(bar_id, kEpiThreads);  // the caller's reads of rows_sm are done
+  if (et < 32) {
+    // compact the columns that hold a slot (ballot + prefix count, in order)
+    int n = 0;
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      const int c = c0 + et;
+      const bool v = c < BN && tok_sm[c] >= 0;
+      const uint32_t mask = __ballot_sync(0xffffffffu, v);
+      if (v) rows_sm[n + __popc(mask & ((1u << et) - 1u))] = c;
+      n += __popc(mask);
+    }
+    if (et == 0) *reinterpret_cast<int*>(inv_sm + BN) = n;
   }
   named_bar_sync(bar_id, kEpiThreads);
-  const int chunks = g.I / 8;  // 8 columns per step: two 16-byte fp32 loads, one 8-byte e4m3 store
-  const int total = BN * chunks;
-  for (int i = et; i < total; i += kEpiThreads) {
-    const int c = i / chunks;
-    const size_t off = static_cast<size_t>(blk * BN + c) * g.I + static_cast<size_t>(i - c * chunks) * 8;
-    const float4 a = __ldcg(reinterpret_cast<const float4*>(g.h32 + off));
-    const float4 b = __ldcg(reinterpret_cast<const float4*>(g.h32 + off + 4));
-    const float sc = scale_sm[c];
-    const uint32_t q0 = cvt_e4m3x2(a.x / sc, a.y / sc), q1 = cvt_e4m3x2(a.z / sc, a.w / sc);
-    const uint32_t q2 = cvt_e4m3x2(b.x / sc, b.y / sc), q3 = cvt_e4m3x2(b.z / sc, b.w / sc);
-    *reinterpret_cast<uint2*>(g.hq + off) = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
+  const int nrows = *reinterpret_cast<const int*>(inv_sm + BN);
+  // row amax from the per-tile partials: TPR threads per row, combined by shuffles
+  constexpr int TPR = BN >= kEpiThreads ? 1 : kEpiThreads / BN;
+  for (int j0 = 0; j0 < nrows; j0 += kEpiThreads / TPR) {
+    const int j = j0 + et / TPR;
+    const int part = et % TPR;
+    const int r = blk * BN + (j < nrows ? rows_sm[j] : 0);
+    float m = 0.f;
+    if (j < nrows) {
+#pragma unroll 4
+      for (int t = part; t < g.n_mt; t += TPR) m = fmaxf(m, __ldcg(g.h_amax + static_cast<size_t>(t) * g.rows_cap + r));
+    }
+#pragma unroll
+    for (int o = TPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (part == 0 && j < nrows) {
+      const float sc = m > 0.f ? m / 448.0f : 1.0f;
+      inv_sm[j] = 1.0f / sc;
+      g.h_scale[r] = sc;
+    }
+  }
+  named_bar_sync(bar_id, kEpiThreads);
+  const int chunks = g.I / 8;  // 8 columns per chunk: two 16-byte fp32 loads, one 8-byte e4m3 store
+  const int total = nrows * chunks;
+  const size_t row0 = static_cast<size_t>(blk) * BN;
+  for (int base = et; base < total; base += kEpiThreads * kQuantUnroll) {
+    float4 a[kQuantUnroll], b[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int i = base + u * kEpiThreads;
+      if (i < total) {
+        const int j = i / chunks;
+        const size_t off = (row0 + rows_sm[j]) * g.I + static_cast<size_t>(i - j * chunks) * 8;
+        a[u] = __ldcg(reinterpret_cast<const float4*>(g.h32 + off));
+        b[u] = __ldcg(reinterpret_cast<const float4*>(g.h32 + off + 4));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int i = base + u * kEpiThreads;
+      if (i < total) {
+        const int j = i / chunks;
+        const size_t off = (row0 + rows_sm[j]) * g.I + static_cast<size_t>(i - j * chunks) * 8;
+        const float iv = inv_sm[j];
+        const uint32_t q0 = cvt_e4m3x2(a[u].x * iv, a[u].y * iv), q1 = cvt_e4m3x2(a[u].z * iv, a[u].w * iv);
+        const uint32_t q2 = cvt_e4m3x2(b[u].x * iv, b[u].y * iv), q3 = cvt_e4m3x2(b[u].z * iv, b[u].w * iv);
+        *reinterpret_cast<uint2*>(g.hq + off) = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
+      }
+    }
   }
 }
 
@@ -271,15 +321,17 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
     bool ok = true;
     // MXFP8 stage 1: gather the token rows' scale bytes of stages [4c, 4c+4)
     // (16 bytes per row) into staging buffer c % 2.
+    // (warp-collective: lane 0 arms the barrier, the lanes issue the row gathers)
     auto issue_stage_scales = [&](int c) {
       const int b = c & 1;
-      fence_proxy_async_smem();  // earlier generic reads of this buffer come first
-      mbar_arrive_expect_tx(&stg_full[b], BN * 16);
-#pragma unroll 4
-      for (int q = 0; q < BN / 4; ++q)
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&stg_full[b], BN * 16);
+        stg_pending |= 1u << b;
+      }
+      __syncwarp();
+      for (int q = lane; q < BN / 4; q += 32)
         tma_gather4(stg + b * L::kStgBuf + q * 128, &tmS, &stg_full[b], c * 16, rows_sm[4 * q],
                     rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
-      stg_pending |= 1u << b;
     };
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const int blk = tile / g.n_mt;
@@ -299,7 +351,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           rows_sm[i] = row;
         }
         __syncwarp();
-        if (MX && lane == 0) issue_stage_scales(0);
+        if (MX) issue_stage_scales(0);
       }
       for (int kb = 0; kb < g.num_kb; ++kb) {
         uint8_t* a_dst = smem + stage * L::kStageBytes;
@@ -309,17 +361,20 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         if (lane == 0) {
           ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
           if (ok && MX && S1 && (kb & 3) == 0) {
-            const int c = kb >> 2, b = c & 1;
+            const int b = (kb >> 2) & 1;
             ok = mbar_wait(&stg_full[b], (stg_phase >> b) & 1u, abort_flag);
             if (ok) {
               stg_phase ^= 1u << b;
               stg_pending &= ~(1u << b);
-              if ((c + 1) * 4 < g.num_kb) issue_stage_scales(c + 1);
             }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        if (MX && S1 && (kb & 3) == 0 && (kb + 4) < g.num_kb) {
+          // the other staging buffer was consumed (and fenced) four stages ago
+          issue_stage_scales((kb >> 2) + 1);
+        }
         if (MX && S1) {
           // this stage's 4 K-block bytes of every token row, into the tile layout
           // (row n sits at byte (n / 4) * 128 + (n % 4) * 16 of its staging buffer)
@@ -337,10 +392,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], bytes);
           if (S1) {
             tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
-#pragma unroll 4
-            for (int q = 0; q < BN / 4; ++q)
-              tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
-                          rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
           } else {
             tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
             tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
@@ -356,6 +407,13 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
         }
         __syncwarp();
+        if (S1) {
+          // token rows, four per gather, issued by the lanes of the warp (the
+          // barrier was armed above with the stage's full byte count)
+          for (int q = lane; q < BN / 4; q += 32)
+            tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
+                        rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -567,7 +625,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
             last_sm[0] = last ? 1 : 0;
           }
           named_bar_sync(bar_id, kEpiThreads);
-          if (last_sm[0]) quantize_block_rows<BN>(g, blk, et, bar_id, amax_part);
+          if (last_sm[0]) quantize_block_rows<BN>(g, blk, et, bar_id, tok_sm, last_sm, amax_part);
         }
       } else {
         const int n = mt * kTileM + 32 * q + lane;  // output feature
