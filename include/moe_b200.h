@@ -108,12 +108,19 @@ size_t moe_sorted_capacity(int T, int top_k, int E, int block_m);
  * zeroes it ONCE after allocating it; each complete call leaves it zeroed. */
 size_t moe_stage2_workspace_bytes(int T, int H);
 
-/* Bytes of the stage-1 workspace for `dtype` (0 when none is needed). For
- * MOE_DT_FP8_E4M3: the unquantised h as fp32, a per-tile row amax and one
- * arrival counter per token block, for `capacity` rows of I columns. The
- * caller zeroes it ONCE after allocating it; each complete call leaves the
+/* Bytes of the stage-1 workspace for `dtype` (0 when none is needed), for
+ * `capacity` rows; 256-byte aligned parts, in this order:
+ *  - MOE_DT_FP8_E4M3: the unquantised h as fp32 [rows, I], a per-tile row
+ *    amax and one arrival counter per token block;
+ *  - block_m >= 32: the token rows of x copied into sorted order [rows, H]
+ *    (x's element type), which the GEMM then reads with one TMA box per
+ *    stage instead of gathering rows four at a time (identity routing reads x
+ *    itself and leaves this part unused);
+ *  - MOE_DT_MXFP8_E4M3: the token scale bytes placed in 512-byte tiles, one
+ *    per (token block, 128 columns of H).
+ * The caller zeroes it ONCE after allocating it; each complete call leaves the
  * counters at zero. */
-size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int I, int block_m);
+size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int I, int block_m);
 
 /* Bytes of the packed MXFP8 weight scales of one projection: which = 0 for W13
  * ([E,2I,H] weights), which = 1 for W2 ([E,H,I] weights). 0 unless H and I are
@@ -188,8 +195,10 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
  *     a  *= x_scale[t] * w13_scale[e]               (MOE_DT_FP8_E4M3; [6106])
  *     h_r = SiLU(a[0:I]) * a[I:2I]
  * then h_r is stored in the stage-2 operand format ([6106]: quantisation fused
- * after the activation). tcgen05 tensor cores, weights streamed by TMA, token
- * rows gathered by TMA.
+ * after the activation). tcgen05 tensor cores, weights streamed by TMA; token
+ * rows gathered by TMA (block_m 16), or copied into sorted order by a
+ * preparation kernel launched first on `stream` (block_m >= 32; MXFP8 token
+ * scales always), then read one box per stage.
  *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3 or MOE_DT_MXFP8_E4M3.
  *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8), ue8m0 bytes
  *              [T,H/32] row-major (MXFP8), or NULL (BF16).
@@ -211,11 +220,12 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
  *              all-zero block) and codes e4m3(h * 2^-X); tile layout as in
  *              moe_mx_pack_weight_scales with the block_m rows of one token
  *              block per tile. NULL for BF16.
- *   ws         FP8: moe_stage1_workspace_bytes(...) bytes, zeroed once by the
- *              caller. NULL for BF16.
- * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8) / % 512 == 0 (MXFP8),
- * I % 64 == 0 (% 128 for MXFP8), block_m in {16,32,64,128,256} (<= 128 for
- * MXFP8), 16-byte aligned x, w13, h, ws and the MXFP8 scale arrays. */
+ *   ws         moe_stage1_workspace_bytes(...) bytes, zeroed once by the
+ *              caller; may be NULL only when that size is 0 (BF16 with
+ *              block_m 16, or BF16 identity routing).
+ * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8, MXFP8), I % 64 == 0 (% 128
+ * for MXFP8), block_m in {16,32,64,128,256} (<= 128 for MXFP8), 16-byte
+ * aligned x, w13, h, ws and the MXFP8 scale arrays. */
 moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, const void* w13,
                              const void* w13_scale, const int32_t* sorted_ids,
                              const int32_t* block_expert, const int32_t* num_padded, int T,

@@ -30,7 +30,7 @@ SIGNATURES = {
     "moe_device_error": (_I, [ctypes.POINTER(ctypes.c_int), _P]),
     "moe_sorted_capacity": (_SZ, [_I, _I, _I, _I]),
     "moe_stage2_workspace_bytes": (_SZ, [_I, _I]),
-    "moe_stage1_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "moe_stage1_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "moe_mx_weight_scale_bytes": (_SZ, [_I, _I, _I, _I]),
     "moe_mx_h_scale_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_mx_pack_weight_scales": (_I, [_I, _P, _P, _I, _I, _I, _P]),
@@ -107,8 +107,8 @@ def stage2_workspace_bytes(T: int, H: int) -> int:
     return lib().moe_stage2_workspace_bytes(T, H)
 
 
-def stage1_workspace_bytes(dtype: int, T: int, top_k: int, E: int, I: int, block_m: int) -> int:
-    return lib().moe_stage1_workspace_bytes(dtype, T, top_k, E, I, block_m)
+def stage1_workspace_bytes(dtype: int, T: int, top_k: int, E: int, H: int, I: int, block_m: int) -> int:
+    return lib().moe_stage1_workspace_bytes(dtype, T, top_k, E, H, I, block_m)
 
 
 def mx_weight_scale_bytes(which: int, E: int, H: int, I: int) -> int:

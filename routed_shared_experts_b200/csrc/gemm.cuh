@@ -41,6 +41,11 @@ constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte s
 constexpr int kEpiThreads = 128;  // one epilogue warpgroup
 constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
 constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)
+// Stage 1 with a sorted token tile of at least this many rows reads its token
+// rows from a copy in sorted order (k_stage1_prep) with one 2-D box per stage:
+// tile::gather4 moves 4 rows per instruction, and at 32 rows per stage the
+// gathers, not HBM, bound the mainloop.
+constexpr int kPermuteMinBN = 32;
 
 enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2 };
 
@@ -60,6 +65,8 @@ struct GemmArgs {
   const int32_t* block_expert;
   const int32_t* num_padded;
   int identity_rows;  // identity routing: rows padded to BN
+  int b_tile;         // stage 1: 1 = token rows are one 2-D box at row blk*BN of tmB (identity routing
+                      // over x, or the sorted copy); 0 = gathered from x four rows per tile::gather4
   int cap_blocks;     // token blocks the sorted buffers can hold
   int T, top_k, H, I;
   int n_mt;    // weight tiles per token block
@@ -77,6 +84,7 @@ struct GemmArgs {
   // MXFP8
   const uint8_t* wsf;  // weight scale tiles [E][n_mt][num_kb][512] (moe_mx_pack_weight_scales)
   uint8_t* hsf;        // h scale tiles [blocks][I/128][512] (stage-1 output, stage-2 input)
+  const uint8_t* xsf;  // stage 1: token scale tiles [blocks][H/128][512] (k_stage1_prep)
   // stage 2
   const void* weights;  // [T*k] or nullptr
   int weights_dtype;    // 4 = f32, 0 = bf16, 1 = fp16
@@ -95,14 +103,9 @@ struct GemmSmem {
   static constexpr int kBBytes = BN * kTileKBytes;
   static constexpr int kSfBytes = kMx ? 2 * kSfTile : 0;  // A then B scale tile
   static constexpr int kStageBytes = kABytes + kBBytes + kSfBytes;
-  // MXFP8 stage 1: token scale bytes gathered 16 per row (4 stages) into two
-  // buffers; each gather of 4 rows (64 bytes) gets its own 128-byte-aligned slot
-  static constexpr int kStgBuf = BN / 4 * 128;
-  static constexpr int kStgBytes = kMx ? 2 * kStgBuf : 0;
-  static constexpr int kStgOffset = STAGES * kStageBytes;
-  static constexpr int kBarOffset = kStgOffset + kStgBytes;
-  // full[S], empty[S], acc_full[A], acc_empty[A], drain, staging[2]
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1 + 2;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  // full[S], empty[S], acc_full[A], acc_empty[A], drain
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
   // tmem slot, abort flag, 2 pad words, producer rows[BN]; then per epilogue
   // group: ok flag + 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
@@ -247,10 +250,59 @@ __device__ __noinline__ void quantize_block_rows(const GemmArgs& g, int blk, int
 // in column n / 32, the four K-block bytes of row n.
 __host__ __device__ constexpr int sf_tile_offset(int n, int kb) { return (n % 32) * 16 + (n / 32) * 4 + kb; }
 
+// Stage-1 operand preparation, run before the GEMM on the same stream.
+// Row r of the sorted order (slot f = sorted_ids[r], token f / top_k; with
+// identity routing token r) gets
+//  * xs: a copy of its token's x row (sorted token tiles of kPermuteMinBN
+//    rows or more), so that the GEMM loads BN rows with one box;
+//  * xsf (MXFP8): its token's ue8m0 scale bytes, placed in the 512-byte tile
+//    of (token block r / bm, stage c) at sf_tile_offset(r % bm, 0..3), the
+//    layout the MMA's scale copy takes, so that the GEMM loads one tile per
+//    stage as it does for the weights.
+// Padding rows are skipped: the MMA column of a padding row is never read.
+struct PrepArgs {
+  const uint8_t* x;           // [T][row_bytes]
+  const uint8_t* x_scale;     // MXFP8: [T][H / 32]
+  const int32_t* sorted_ids;  // nullptr: identity routing
+  const int32_t* num_padded;
+  int identity_rows, rows_cap, T, top_k, row_bytes, H, bm;
+  uint8_t* xs;   // [rows_cap][row_bytes] or nullptr
+  uint8_t* xsf;  // [rows_cap / bm][H / 128][512] or nullptr
+};
+constexpr int kPrepWarps = 8;
+__global__ void __launch_bounds__(kPrepWarps * 32) k_stage1_prep(const PrepArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int rows = a.sorted_ids ? *a.num_padded : a.identity_rows;
+  if (rows > a.rows_cap) rows = a.rows_cap;
+  const int slots = a.T * a.top_k;
+  const int stages = a.H / 128;
+  for (int r = blockIdx.x * kPrepWarps + warp; r < rows; r += gridDim.x * kPrepWarps) {
+    int t = -1;
+    if (!a.sorted_ids) {
+      if (r < a.T) t = r;
+    } else {
+      const int f = a.sorted_ids[r];
+      if (f >= 0 && f < slots) t = f / a.top_k;
+    }
+    if (t < 0) continue;
+    if (a.xs) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.row_bytes);
+      uint4* dst = reinterpret_cast<uint4*>(a.xs + static_cast<size_t>(r) * a.row_bytes);
+      for (int i = lane; i < a.row_bytes / 16; i += 32) dst[i] = __ldg(src + i);
+    }
+    if (a.xsf) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(a.x_scale + static_cast<size_t>(t) * (a.H / 32));
+      const int blk = r / a.bm;
+      uint8_t* tiles = a.xsf + static_cast<size_t>(blk) * stages * kSfTile + sf_tile_offset(r - blk * a.bm, 0);
+      for (int c = lane; c < stages; c += 32) *reinterpret_cast<uint32_t*>(tiles + static_cast<size_t>(c) * kSfTile) = src[c];
+    }
+  }
+}
+
 template <int BN, int STAGES, bool S1, int KIND>
 __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
-    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmS, const GemmArgs g) {
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
   using L = GemmSmem<BN, STAGES, KIND>;
   constexpr bool FP8 = KIND == kFp8;
   constexpr bool MX = KIND == kMx8;
@@ -270,8 +322,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* drain = acc_empty + NACC;
-  uint64_t* stg_full = drain + 1;  // MXFP8 stage 1: token-scale staging buffers
-  uint8_t* stg = smem + L::kStgOffset;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* rows_sm = reinterpret_cast<int*>(tmem_slot + 4);
@@ -290,8 +340,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
       mbar_init(&acc_empty[a], kEpiThreads);
     }
     mbar_init(drain, 1);
-    mbar_init(&stg_full[0], 1);
-    mbar_init(&stg_full[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -316,82 +364,38 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t pending = 0, pend_parity = 0;  // stages armed and not yet re-acquired
-    uint32_t stg_phase = 0;                 // MXFP8 stage 1: parity bits of the two staging buffers
-    uint32_t stg_pending = 0;
     bool ok = true;
-    // MXFP8 stage 1: gather the token rows' scale bytes of stages [4c, 4c+4)
-    // (16 bytes per row) into staging buffer c % 2.
-    // (warp-collective: lane 0 arms the barrier, the lanes issue the row gathers)
-    auto issue_stage_scales = [&](int c) {
-      const int b = c & 1;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&stg_full[b], BN * 16);
-        stg_pending |= 1u << b;
-      }
-      __syncwarp();
-      for (int q = lane; q < BN / 4; q += 32)
-        tma_gather4(stg + b * L::kStgBuf + q * 128, &tmS, &stg_full[b], c * 16, rows_sm[4 * q],
-                    rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
-    };
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const int blk = tile / g.n_mt;
       const int mt = tile - blk * g.n_mt;
       const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
-      if (S1) {
+      if (S1 && !g.b_tile) {
         for (int i = lane; i < BN; i += 32) {
           const int r = blk * BN + i;
           int row = 0;
-          if (!g.sorted_ids) {
-            row = r < g.T ? r : 0;
-          } else {
-            const int f = g.sorted_ids[r];
-            if (f >= 0 && f < slots) row = f / g.top_k;
-            else if (f != slots) set_device_error(kErrSlotRange);
-          }
+          const int f = g.sorted_ids[r];
+          if (f >= 0 && f < slots) row = f / g.top_k;
+          else if (f != slots) set_device_error(kErrSlotRange);
           rows_sm[i] = row;
         }
         __syncwarp();
-        if (MX) issue_stage_scales(0);
       }
       for (int kb = 0; kb < g.num_kb; ++kb) {
         uint8_t* a_dst = smem + stage * L::kStageBytes;
         uint8_t* b_dst = a_dst + L::kABytes;
         uint8_t* sfa_dst = b_dst + L::kBBytes;
         uint8_t* sfb_dst = sfa_dst + kSfTile;
-        if (lane == 0) {
-          ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
-          if (ok && MX && S1 && (kb & 3) == 0) {
-            const int b = (kb >> 2) & 1;
-            ok = mbar_wait(&stg_full[b], (stg_phase >> b) & 1u, abort_flag);
-            if (ok) {
-              stg_phase ^= 1u << b;
-              stg_pending &= ~(1u << b);
-            }
-          }
-        }
+        if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        if (MX && S1 && (kb & 3) == 0 && (kb + 4) < g.num_kb) {
-          // the other staging buffer was consumed (and fenced) four stages ago
-          issue_stage_scales((kb >> 2) + 1);
-        }
-        if (MX && S1) {
-          // this stage's 4 K-block bytes of every token row, into the tile layout
-          // (row n sits at byte (n / 4) * 128 + (n % 4) * 16 of its staging buffer)
-          const uint32_t* src = reinterpret_cast<const uint32_t*>(stg + ((kb >> 2) & 1) * L::kStgBuf);
-          uint32_t* dst = reinterpret_cast<uint32_t*>(sfb_dst);
-          for (int n = lane; n < BN; n += 32)
-            dst[sf_tile_offset(n, 0) / 4] = src[(n / 4) * 32 + (n % 4) * 4 + (kb & 3)];
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
         if (lane == 0) {
           pending &= ~(1u << stage);
           uint32_t bytes = L::kABytes + L::kBBytes;
-          if (MX) bytes += S1 ? kSfTile : 2 * kSfTile;
+          if (MX) bytes += 2 * kSfTile;
           mbar_arrive_expect_tx(&full[stage], bytes);
           if (S1) {
             tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+            if (g.b_tile) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
           } else {
             tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
             tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
@@ -399,15 +403,14 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           if (MX) {
             const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
             bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
-            if (!S1)
-              bulk_load(sfb_dst, g.hsf + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile, kSfTile,
-                        &full[stage], pol_x);
+            bulk_load(sfb_dst, (S1 ? g.xsf : g.hsf) + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile,
+                      kSfTile, &full[stage], pol_x);
           }
           pending |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
         }
         __syncwarp();
-        if (S1) {
+        if (S1 && !g.b_tile) {
           // token rows, four per gather, issued by the lanes of the warp (the
           // barrier was armed above with the stage's full byte count)
           for (int q = lane; q < BN / 4; q += 32)
@@ -424,8 +427,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
     if (!ok && lane == 0) {
       for (int s = 0; s < STAGES; ++s)
         if ((pending >> s) & 1u) drain_wait(&full[s], (pend_parity >> s) & 1u);
-      for (int b = 0; b < 2; ++b)
-        if ((stg_pending >> b) & 1u) drain_wait(&stg_full[b], (stg_phase >> b) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -96,15 +96,16 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
 template <int BN, int KIND>
 constexpr int stages_for() {
   // as many stages as fit in 227 KB of shared memory, one CTA per SM
-  if (KIND == moe::kMx8) return BN == 16 ? 10 : BN == 32 ? 9 : BN == 64 ? 7 : 5;
-  return BN == 16 ? 12 : BN == 32 ? 11 : BN == 64 ? 8 : BN == 128 ? 6 : 4;
+  if (KIND == moe::kMx8) return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : 6;
+  return BN == 16 ? 12 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
 }
 
 template <int BN, bool S1, int KIND>
-moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
-                            const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
+moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
+                            cudaStream_t s) {
   constexpr int ST = stages_for<BN, KIND>();
   using L = moe::GemmSmem<BN, ST, KIND>;
+  static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
   auto kern = moe::k_moe_gemm<BN, ST, S1, KIND>;
   static std::atomic<int> attr_set[64];
   int dev = 0;
@@ -115,32 +116,32 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
   }
   int grid = max_tiles < num_sms() ? max_tiles : num_sms();
   if (grid < 1) grid = 1;
-  kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, ts, g);
+  kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, g);
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
 
 template <bool S1, int KIND>
-moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
-                         const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
+moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
+                         cudaStream_t s) {
   switch (bm) {
-    case 16: return launch_gemm_bn<16, S1, KIND>(ta, tb, ts, g, max_tiles, s);
-    case 32: return launch_gemm_bn<32, S1, KIND>(ta, tb, ts, g, max_tiles, s);
-    case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, ts, g, max_tiles, s);
-    case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+    case 16: return launch_gemm_bn<16, S1, KIND>(ta, tb, g, max_tiles, s);
+    case 32: return launch_gemm_bn<32, S1, KIND>(ta, tb, g, max_tiles, s);
+    case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, g, max_tiles, s);
+    case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, g, max_tiles, s);
     case 256:
-      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, ts, g, max_tiles, s);
+      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, g, max_tiles, s);
       break;
   }
   return MOE_ERR_INVALID_ARG;
 }
 
 template <bool S1>
-moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
-                              const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
-  if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, ts, g, max_tiles, s);
-  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, ts, g, max_tiles, s);
-  return launch_gemm<S1, moe::kBf16>(bm, ta, tb, ts, g, max_tiles, s);
+moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g,
+                              int max_tiles, cudaStream_t s) {
+  if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, g, max_tiles, s);
+  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, g, max_tiles, s);
+  return launch_gemm<S1, moe::kBf16>(bm, ta, tb, g, max_tiles, s);
 }
 
 // Padded sorted length bound T*k + E*(bm-1), rounded up to whole blocks.
@@ -149,15 +150,26 @@ size_t capacity(int T, int k, int E, int bm) {
   return (n + bm - 1) / bm * bm;
 }
 
-// Stage-1 workspace of the fp8 path: unquantised fp32 h [rows, I], per-tile
-// row amax [I/64][rows], one arrival counter per token block; 256-byte aligned parts.
+// Stage-1 workspace, 256-byte aligned parts:
+//  * fp8: unquantised fp32 h [rows, I], per-tile row amax [I/64][rows], one
+//    arrival counter per token block;
+//  * block_m >= kPermuteMinBN: token rows in sorted order [rows, H] (x's type);
+//  * MXFP8: token scale tiles [rows / block_m][H / 128][512].
 struct Stage1Ws {
-  size_t amax_off, cnt_off, total;
-  Stage1Ws(size_t rows, int I, int bm) {
+  size_t amax_off = 0, cnt_off = 0, xs_off = 0, xsf_off = 0, total = 0;
+  Stage1Ws(int dtype, size_t rows, int H, int I, int bm) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-    amax_off = up(rows * static_cast<size_t>(I) * 4);
-    cnt_off = amax_off + up(static_cast<size_t>((I + 63) / 64) * rows * 4);
-    total = cnt_off + up(rows / bm * 4);
+    size_t o = 0;
+    if (dtype == MOE_DT_FP8_E4M3) {
+      amax_off = up(rows * static_cast<size_t>(I) * 4);
+      cnt_off = amax_off + up(static_cast<size_t>((I + 63) / 64) * rows * 4);
+      o = cnt_off + up(rows / bm * 4);
+    }
+    xs_off = o;
+    if (bm >= moe::kPermuteMinBN) o += up(rows * static_cast<size_t>(H) * (dtype == MOE_DT_BF16 ? 2 : 1));
+    xsf_off = o;
+    if (dtype == MOE_DT_MXFP8_E4M3) o += up(rows / bm * static_cast<size_t>(H / 128) * moe::kSfTile);
+    total = o;
   }
 };
 
@@ -233,9 +245,10 @@ size_t moe_stage2_workspace_bytes(int T, int H) {
   return static_cast<size_t>(T) * H * sizeof(float) + static_cast<size_t>(T) * n_mt * sizeof(int);
 }
 
-size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int I, int block_m) {
-  if (dtype != MOE_DT_FP8_E4M3 || T < 1 || top_k < 1 || E < 1 || I < 1 || !valid_block_m(block_m)) return 0;
-  return Stage1Ws(capacity(T, top_k, E, block_m), I, block_m).total;
+size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int I, int block_m) {
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && dtype != MOE_DT_MXFP8_E4M3) return 0;
+  if (T < 1 || top_k < 1 || E < 1 || H < 1 || I < 1 || !valid_block_m(block_m)) return 0;
+  return Stage1Ws(dtype, capacity(T, top_k, E, block_m), H, I, block_m).total;
 }
 
 moe_status_t moe_router_topk(const float* logits, const float* correction_bias, int T, int E, int top_k, int mode,
@@ -321,11 +334,14 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  if (fp8 && (!x_scale || !w13_scale || !h_scale || !ws)) return MOE_ERR_INVALID_ARG;
+  // routed tiles of kPermuteMinBN rows or more read a sorted copy of the token rows
+  const bool permute = sorted_ids && block_m >= moe::kPermuteMinBN;
+  if (fp8 && (!x_scale || !w13_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
   if (mx && (!x_scale || !w13_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+  if ((fp8 || mx || permute) && !ws) return MOE_ERR_INVALID_ARG;
   if (mx && block_m > 128) return MOE_ERR_INVALID_ARG;
   if (H % (dtype == MOE_DT_BF16 ? 64 : 128) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
-  if (mx && (H % 512 != 0 || I % 128 != 0)) return MOE_ERR_ALIGNMENT;  // whole 16-byte scale runs, 4-block tiles
+  if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;  // whole 4-block h scale tiles
   if (!aligned16(x) || !aligned16(w13) || !aligned16(h) || (ws && !aligned16(ws)) ||
       (mx && (!aligned16(x_scale) || !aligned16(w13_scale) || !aligned16(h_scale))))
     return MOE_ERR_ALIGNMENT;
@@ -341,7 +357,11 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   // W13 as 5-D (K, row-in-16, gate|up, 16-row group, expert): one box brings
   // 16 gate rows then the 16 matching up rows for four consecutive groups, so
   // the 128 weight rows of a tile pair gate and up inside each 32-lane quarter.
-  CUtensorMap ta, tb, ts;
+  const Stage1Ws L(dtype, rows_cap, H, I, block_m);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint8_t* xs = permute ? wsb + L.xs_off : nullptr;
+  uint8_t* xsf = mx ? wsb + L.xsf_off : nullptr;
+  CUtensorMap ta, tb;
   {
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(H), 16, 2, static_cast<cuuint64_t>(I / 16),
                                 static_cast<cuuint64_t>(E)};
@@ -352,20 +372,15 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     if (r != MOE_OK) return r;
   }
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    // token rows: one [block_m x 128 B] box per stage from x (identity
+    // routing; rows past T read as zeros) or from the sorted copy; else
+    // single rows of x for tile::gather4
+    const bool tile = permute || !sorted_ids;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), permute ? static_cast<cuuint64_t>(rows_cap)
+                                                                    : static_cast<cuuint64_t>(T)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), 1};
-    moe_status_t r = make_map(&tb, tdt, 2, x, dims, st, box);
-    if (r != MOE_OK) return r;
-  }
-  ts = tb;
-  if (mx) {
-    // token scale bytes [T][H/32], gathered 16 bytes (4 stages) per row
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H / 32), static_cast<cuuint64_t>(T)};
-    const cuuint64_t st[1] = {static_cast<cuuint64_t>(H / 32)};
-    const cuuint32_t box[2] = {16, 1};
-    moe_status_t r = make_map(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, x_scale, dims, st, box,
-                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), tile ? static_cast<cuuint32_t>(block_m) : 1u};
+    moe_status_t r = make_map(&tb, tdt, 2, permute ? static_cast<const void*>(xs) : x, dims, st, box);
     if (r != MOE_OK) return r;
   }
   moe::GemmArgs g{};
@@ -373,6 +388,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   g.block_expert = block_expert;
   g.num_padded = num_padded;
   g.identity_rows = cap_blocks * block_m;
+  g.b_tile = (permute || !sorted_ids) ? 1 : 0;
   g.cap_blocks = cap_blocks;
   g.T = T;
   g.top_k = top_k;
@@ -382,11 +398,9 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   g.num_kb = H / ke;
   g.rows_cap = static_cast<int>(rows_cap);
   if (fp8) {
-    const Stage1Ws L(rows_cap, I, block_m);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    g.h32 = reinterpret_cast<float*>(w);
-    g.h_amax = reinterpret_cast<float*>(w + L.amax_off);
-    g.blk_cnt = reinterpret_cast<int*>(w + L.cnt_off);
+    g.h32 = reinterpret_cast<float*>(wsb);
+    g.h_amax = reinterpret_cast<float*>(wsb + L.amax_off);
+    g.blk_cnt = reinterpret_cast<int*>(wsb + L.cnt_off);
     g.hq = static_cast<uint8_t*>(h);
     g.h_scale = static_cast<float*>(h_scale);
     g.x_scale = static_cast<const float*>(x_scale);
@@ -395,11 +409,33 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     g.hq = static_cast<uint8_t*>(h);
     g.hsf = static_cast<uint8_t*>(h_scale);
     g.wsf = static_cast<const uint8_t*>(w13_scale);
+    g.xsf = xsf;
   } else {
     g.h = static_cast<__nv_bfloat16*>(h);
   }
+  cudaStream_t s = as_stream(stream);
+  if (xs || xsf) {
+    moe::PrepArgs p{};
+    p.x = static_cast<const uint8_t*>(x);
+    p.x_scale = static_cast<const uint8_t*>(x_scale);
+    p.sorted_ids = sorted_ids;
+    p.num_padded = num_padded;
+    p.identity_rows = g.identity_rows;
+    p.rows_cap = static_cast<int>(rows_cap);
+    p.T = T;
+    p.top_k = top_k;
+    p.row_bytes = H * es;
+    p.H = H;
+    p.bm = block_m;
+    p.xs = xs;
+    p.xsf = xsf;
+    const size_t want = (rows_cap + moe::kPrepWarps - 1) / moe::kPrepWarps;
+    const int grid = static_cast<int>(want < 16u * num_sms() ? want : 16u * num_sms());
+    moe::k_stage1_prep<<<grid, moe::kPrepWarps * 32, 0, s>>>(p);
+    MOE_CK(cudaGetLastError());
+  }
   const int max_tiles = cap_blocks * g.n_mt;
-  return launch_gemm_kind<true>(dtype, block_m, ta, tb, ts, g, max_tiles, as_stream(stream));
+  return launch_gemm_kind<true>(dtype, block_m, ta, tb, g, max_tiles, s);
 }
 
 moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale, const void* w2,
@@ -480,7 +516,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
-  return launch_gemm_kind<false>(dtype, block_m, ta, tb, tb, g, max_tiles, s);
+  return launch_gemm_kind<false>(dtype, block_m, ta, tb, g, max_tiles, s);
 }
 
 size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I) {

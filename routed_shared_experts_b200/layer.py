@@ -69,8 +69,8 @@ class MoELayer:
                 self.wsc[name] = dst
             else:
                 self.wsc[name] = inp.get(name + "_scale")
-        ws1 = capi.stage1_workspace_bytes(self.dt, T, k, E, I, bm)
-        ws1s = capi.stage1_workspace_bytes(self.dt, T, 1, 1, Is, bm)
+        ws1 = capi.stage1_workspace_bytes(self.dt, T, k, E, H, I, bm)
+        ws1s = capi.stage1_workspace_bytes(self.dt, T, 1, 1, H, Is, bm)
         self.ws1 = torch.zeros(ws1, dtype=torch.uint8, device=dev) if ws1 else None  # zeroed once
         self.ws1_s = torch.zeros(ws1s, dtype=torch.uint8, device=dev) if ws1s else None
         gdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float16

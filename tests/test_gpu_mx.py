@@ -77,6 +77,14 @@ def test_mx_random_scales(cuda_lib, block_m):
     _check(SMALL_MX, _inputs(SMALL_MX), block_m=block_m)
 
 
+@pytest.mark.parametrize("block_m", [16, 128])
+def test_mx_hidden_not_multiple_of_512(cuda_lib, block_m):
+    """H = 640: five 128-column K stages per tile, so the token scale tiles of
+    stage 1 do not come in groups of four stages."""
+    cfg = configs.small(SMALL_MX, name="small_mx_h640", H=640, seed=33)
+    _check(cfg, _inputs(cfg), block_m=block_m)
+
+
 def test_mx_prefill_layer(cuda_lib):
     cfg = configs.MXFP8_PREFILL
     inp = synth.make_layer_inputs(cfg, device="cuda")
