@@ -41,6 +41,7 @@ constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte s
 constexpr int kEpiThreads = 128;  // one epilogue warpgroup
 constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
 constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)
+constexpr int kFinBatch = 8;      // stage-2 finalisation: token columns per batch of loads
 // Stage 1 with a sorted token tile of at least this many rows reads its token
 // rows from a copy in sorted order (k_stage1_prep) with one 2-D box per stage:
 // tile::gather4 moves 4 rows per instruction, and at 32 rows per stage the
@@ -673,14 +674,44 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
             }
             last_sm[c] = flag;
           }
+          // Finalise the columns this group brought last: their tokens' sums
+          // are complete (acquired above). The columns are compacted first so
+          // that each thread has kFinBatch independent loads in flight (one L2
+          // round trip per batch instead of one per column).
           named_bar_sync(bar_id, kEpiThreads);
+          int* list = reinterpret_cast<int*>(amax_part);  // BN column indices, then the count
+          if (et < 32) {
+            int cnt = 0;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+              const int c = c0 + et;
+              const bool v = c < BN && last_sm[c];
+              const uint32_t mask = __ballot_sync(0xffffffffu, v);
+              if (v) list[cnt + __popc(mask & ((1u << et) - 1u))] = c;
+              cnt += __popc(mask);
+            }
+            if (et == 0) list[BN] = cnt;
+          }
+          named_bar_sync(bar_id, kEpiThreads);
+          const int nlast = list[BN];
           if (nvalid) {
-            for (int c = 0; c < BN; ++c) {
-              if (!last_sm[c]) continue;
-              const size_t o = static_cast<size_t>(tok_sm[c]) * g.H + n;
-              float y = atomicExch(g.ws + o, 0.0f);
-              if (g.addend) y += __bfloat162float(g.addend[o]);
-              g.out[o] = __float2bfloat16_rn(y);
+            for (int j0 = 0; j0 < nlast; j0 += kFinBatch) {
+              float y[kFinBatch], a[kFinBatch];
+              size_t o[kFinBatch];
+#pragma unroll
+              for (int u = 0; u < kFinBatch; ++u) {
+                if (j0 + u < nlast) {
+                  o[u] = static_cast<size_t>(tok_sm[list[j0 + u]]) * g.H + n;
+                  y[u] = __ldcg(g.ws + o[u]);
+                  a[u] = g.addend ? __bfloat162float(g.addend[o[u]]) : 0.0f;
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < kFinBatch; ++u) {
+                if (j0 + u < nlast) {
+                  __stcg(g.ws + o[u], 0.0f);  // the workspace is left zeroed for the next call
+                  g.out[o[u]] = __float2bfloat16_rn(y[u] + a[u]);
+                }
+              }
             }
           }
         }
