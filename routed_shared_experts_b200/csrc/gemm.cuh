@@ -77,6 +77,9 @@ struct GemmArgs {
   float* h32;        // fp8: the unquantised h [rows, I] in fp32 (workspace)
   float* h_amax;     // fp8: per-tile row amax [n_mt][rows_cap] (workspace)
   int* blk_cnt;      // fp8: finished weight tiles per token block (workspace, self-cleaning)
+  int quant_phase;   // fp8: 1 = rows are quantised after a grid barrier by every warp (cooperative
+                     // launch); 0 = by the epilogue that finishes a token block's last tile
+  unsigned* grid_bar;  // fp8 quant_phase: arrival count, generation (workspace, self-cleaning)
   uint8_t* hq;       // fp8 / MXFP8: e4m3 codes of h [rows, I]
   int rows_cap;
   const float* x_scale;  // fp8: [T]
@@ -108,7 +111,7 @@ struct GemmSmem {
   // full[S], empty[S], acc_full[A], acc_empty[A], drain
   static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
-  // tmem slot, abort flag, 2 pad words, producer rows[BN]; then per epilogue
+  // tmem slot, abort flag, grid-barrier flag, pad word, producer rows[BN]; then per epilogue
   // group: ok flag + 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
   static constexpr int kGroupWords = 4 + 7 * BN;
   static constexpr int kMiscBytes = 16 + BN * 4 + kGroups * kGroupWords * 4;
@@ -297,6 +300,87 @@ __global__ void __launch_bounds__(kPrepWarps * 32) k_stage1_prep(const PrepArgs 
       const int blk = r / a.bm;
       uint8_t* tiles = a.xsf + static_cast<size_t>(blk) * stages * kSfTile + sf_tile_offset(r - blk * a.bm, 0);
       for (int c = lane; c < stages; c += 32) *reinterpret_cast<uint32_t*>(tiles + static_cast<size_t>(c) * kSfTile) = src[c];
+    }
+  }
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier over all CTAs of a cooperative launch (every CTA is resident, so
+// the wait ends once each CTA has arrived). bar[0] counts arrivals and is
+// reset by the last arrival, which then advances the generation bar[1]; the
+// others wait for the generation to move. The wait is bounded: on timeout
+// it records kErrWaitTimeout and returns false. Called by all threads.
+__device__ bool grid_barrier(unsigned* bar, int* flag_sm) {
+  if (threadIdx.x == 0) {
+    const unsigned gen = ld_acquire_gpu(bar + 1);
+    __threadfence();  // this CTA's writes (ordered before by the caller's __syncthreads) first
+    int ok = 1;
+    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (ld_acquire_gpu(bar + 1) == gen) {
+        if (globaltimer() - t0 > kWaitTimeoutNs) {
+          set_device_error(kErrWaitTimeout);
+          ok = 0;
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    *flag_sm = ok;
+  }
+  __syncthreads();
+  return *flag_sm != 0;
+}
+
+// fp8 stage 1, quant_phase: after every weight tile of every token block is
+// done, each warp of the grid quantises whole rows of h (the rows holding a
+// slot; padding rows are never read): row amax over the per-tile partials,
+// s = amax / 448 (amax = 0 -> s = 1), codes e4m3(h * (1 / s)).
+__device__ void quantize_rows_grid(const GemmArgs& g, int rows) {
+  const int lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const int slots = g.T * g.top_k;
+  const int chunks = g.I / 8;  // 8 columns per chunk
+  for (int r = blockIdx.x * nw + (threadIdx.x >> 5); r < rows; r += gridDim.x * nw) {
+    const bool valid = g.sorted_ids ? (static_cast<unsigned>(g.sorted_ids[r]) < static_cast<unsigned>(slots)) : (r < g.T);
+    if (!valid) continue;
+    float m = 0.f;
+    for (int t = lane; t < g.n_mt; t += 32) m = fmaxf(m, __ldcg(g.h_amax + static_cast<size_t>(t) * g.rows_cap + r));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sc = m > 0.f ? m / 448.0f : 1.0f;
+    const float iv = 1.0f / sc;
+    if (lane == 0) g.h_scale[r] = sc;
+    const float* src = g.h32 + static_cast<size_t>(r) * g.I;
+    uint8_t* dst = g.hq + static_cast<size_t>(r) * g.I;
+    for (int base = lane; base < chunks; base += 32 * kQuantUnroll) {
+      float4 a[kQuantUnroll], b[kQuantUnroll];
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int i = base + 32 * u;
+        if (i < chunks) {
+          a[u] = __ldcg(reinterpret_cast<const float4*>(src) + 2 * i);
+          b[u] = __ldcg(reinterpret_cast<const float4*>(src) + 2 * i + 1);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const int i = base + 32 * u;
+        if (i < chunks) {
+          const uint32_t q0 = cvt_e4m3x2(a[u].x * iv, a[u].y * iv), q1 = cvt_e4m3x2(a[u].z * iv, a[u].w * iv);
+          const uint32_t q2 = cvt_e4m3x2(b[u].x * iv, b[u].y * iv), q3 = cvt_e4m3x2(b[u].z * iv, b[u].w * iv);
+          reinterpret_cast<uint2*>(dst)[i] = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
+        }
+      }
     }
   }
 }
@@ -619,15 +703,17 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           // fused after the activation). The barrier orders this group's h and
           // amax stores before the counter's release; the acquire of the last
           // arrival makes every tile's stores visible.
-          named_bar_sync(bar_id, kEpiThreads);
-          if (et == 0) {
-            int* cnt = g.blk_cnt + blk;
-            const bool last = atom_add_acq_rel_gpu(cnt, 1) == g.n_mt - 1;
-            if (last) *cnt = 0;
-            last_sm[0] = last ? 1 : 0;
+          if (!g.quant_phase) {
+            named_bar_sync(bar_id, kEpiThreads);
+            if (et == 0) {
+              int* cnt = g.blk_cnt + blk;
+              const bool last = atom_add_acq_rel_gpu(cnt, 1) == g.n_mt - 1;
+              if (last) *cnt = 0;
+              last_sm[0] = last ? 1 : 0;
+            }
+            named_bar_sync(bar_id, kEpiThreads);
+            if (last_sm[0]) quantize_block_rows<BN>(g, blk, et, bar_id, tok_sm, last_sm, amax_part);
           }
-          named_bar_sync(bar_id, kEpiThreads);
-          if (last_sm[0]) quantize_block_rows<BN>(g, blk, et, bar_id, tok_sm, last_sm, amax_part);
         }
       } else {
         const int n = mt * kTileM + 32 * q + lane;  // output feature
@@ -725,6 +811,10 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+  if constexpr (FP8 && S1) {
+    if (g.quant_phase && grid_barrier(g.grid_bar, reinterpret_cast<int*>(tmem_slot + 2)))
+      quantize_rows_grid(g, n_blocks * BN);
   }
 }
 

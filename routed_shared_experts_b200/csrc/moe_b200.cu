@@ -116,7 +116,14 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
   }
   int grid = max_tiles < num_sms() ? max_tiles : num_sms();
   if (grid < 1) grid = 1;
-  kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, g);
+  if (g.quant_phase) {
+    // every CTA resident at once (one per SM): the grid barrier's wait ends
+    void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<moe::GemmArgs*>(&g)};
+    MOE_CK(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
+                                       dim3(moe::EpiCfg<BN, KIND>::kThreads), args, L::kBytes, s));
+  } else {
+    kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, g);
+  }
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
@@ -152,18 +159,19 @@ size_t capacity(int T, int k, int E, int bm) {
 
 // Stage-1 workspace, 256-byte aligned parts:
 //  * fp8: unquantised fp32 h [rows, I], per-tile row amax [I/64][rows], one
-//    arrival counter per token block;
+//    arrival counter per token block, the grid barrier's two words;
 //  * block_m >= kPermuteMinBN: token rows in sorted order [rows, H] (x's type);
 //  * MXFP8: token scale tiles [rows / block_m][H / 128][512].
 struct Stage1Ws {
-  size_t amax_off = 0, cnt_off = 0, xs_off = 0, xsf_off = 0, total = 0;
+  size_t amax_off = 0, cnt_off = 0, bar_off = 0, xs_off = 0, xsf_off = 0, total = 0;
   Stage1Ws(int dtype, size_t rows, int H, int I, int bm) {
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     size_t o = 0;
     if (dtype == MOE_DT_FP8_E4M3) {
       amax_off = up(rows * static_cast<size_t>(I) * 4);
       cnt_off = amax_off + up(static_cast<size_t>((I + 63) / 64) * rows * 4);
-      o = cnt_off + up(rows / bm * 4);
+      bar_off = cnt_off + up(rows / bm * 4);
+      o = bar_off + 256;
     }
     xs_off = o;
     if (bm >= moe::kPermuteMinBN) o += up(rows * static_cast<size_t>(H) * (dtype == MOE_DT_BF16 ? 2 : 1));
@@ -401,6 +409,10 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     g.h32 = reinterpret_cast<float*>(wsb);
     g.h_amax = reinterpret_cast<float*>(wsb + L.amax_off);
     g.blk_cnt = reinterpret_cast<int*>(wsb + L.cnt_off);
+    g.grid_bar = reinterpret_cast<unsigned*>(wsb + L.bar_off);
+    // token blocks of 64 rows or more hold up to ~1.4 MB of fp32 h each: too
+    // much for one warpgroup, so every warp quantises rows after a grid barrier
+    g.quant_phase = block_m >= 64 ? 1 : 0;
     g.hq = static_cast<uint8_t*>(h);
     g.h_scale = static_cast<float*>(h_scale);
     g.x_scale = static_cast<const float*>(x_scale);

@@ -46,16 +46,17 @@ def test_info_calls(lib):
     assert lib.moe_sorted_capacity(5, 3, 7, 64) == 512  # 15 + 441 = 456 -> 512
     assert lib.moe_stage2_workspace_bytes(32, 2048) == 32 * 2048 * 4 + 32 * 16 * 4
     # stage-1 workspace, 256-byte aligned parts: fp8 fp32 h + per-tile amax +
-    # block counters; sorted token rows when block_m >= 32; MXFP8 token scale tiles
+    # block counters + grid barrier; sorted token rows when block_m >= 32; MXFP8
+    # token scale tiles
     rows = lib.moe_sorted_capacity(1024, 6, 64, 128)
     up = lambda v: (v + 255) // 256 * 256  # noqa: E731
-    want = up(rows * 1408 * 4) + up(22 * rows * 4) + up(rows // 128 * 4) + up(rows * 4096)
+    want = up(rows * 1408 * 4) + up(22 * rows * 4) + up(rows // 128 * 4) + 256 + up(rows * 4096)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 1024, 6, 64, 4096, 1408, 128) == want
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 1024, 6, 64, 4096, 1408, 128) == up(rows * 4096 * 2)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 32, 8, 128, 2048, 768, 16) == 0
     rows16 = lib.moe_sorted_capacity(32, 8, 128, 16)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 32, 8, 128, 2048, 768, 16) == \
-        up(rows16 * 768 * 4) + up(12 * rows16 * 4) + up(rows16 // 16 * 4)
+        up(rows16 * 768 * 4) + up(12 * rows16 * 4) + up(rows16 // 16 * 4) + 256
     rows_mx = lib.moe_sorted_capacity(4096, 8, 256, 128)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_MXFP8_E4M3, 4096, 8, 256, 7168, 2048, 128) == \
         up(rows_mx * 7168) + up(rows_mx // 128 * 56 * 512)
