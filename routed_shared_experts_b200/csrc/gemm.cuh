@@ -780,16 +780,26 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           named_bar_sync(bar_id, kEpiThreads);
           const int nlast = list[BN];
           if (nvalid) {
+            const __nv_bfloat16* add = g.addend;
             for (int j0 = 0; j0 < nlast; j0 += kFinBatch) {
+              // addresses of the batch (a past-the-end entry repeats column
+              // j0 and is loaded but not stored), then all workspace loads,
+              // then all addend loads, then the stores
               float y[kFinBatch], a[kFinBatch];
               size_t o[kFinBatch];
 #pragma unroll
               for (int u = 0; u < kFinBatch; ++u) {
-                if (j0 + u < nlast) {
-                  o[u] = static_cast<size_t>(tok_sm[list[j0 + u]]) * g.H + n;
-                  y[u] = __ldcg(g.ws + o[u]);
-                  a[u] = g.addend ? __bfloat162float(g.addend[o[u]]) : 0.0f;
-                }
+                o[u] = static_cast<size_t>(tok_sm[list[j0 + u < nlast ? j0 + u : j0]]) * g.H + n;
+                y[u] = 0.f;
+                a[u] = 0.f;
+              }
+#pragma unroll
+              for (int u = 0; u < kFinBatch; ++u)
+                if (j0 + u < nlast) y[u] = __ldcg(g.ws + o[u]);
+              if (add) {
+#pragma unroll
+                for (int u = 0; u < kFinBatch; ++u)
+                  if (j0 + u < nlast) a[u] = __bfloat162float(add[o[u]]);
               }
 #pragma unroll
               for (int u = 0; u < kFinBatch; ++u) {
