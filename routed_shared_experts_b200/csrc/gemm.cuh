@@ -304,6 +304,27 @@ __global__ void __launch_bounds__(kPrepWarps * 32) k_stage1_prep(const PrepArgs 
   }
 }
 
+// Token columns of block `blk` that the tile computes: its rows that hold a
+// slot, rounded up to 16 (a valid MMA N; at least 16). The slot rows of a
+// sorted block are a prefix, since the sort puts each expert's padding after
+// its slots; with identity routing they are the rows below T. Warp-collective.
+template <int BN>
+__device__ __forceinline__ int block_cols(const GemmArgs& g, int blk, int lane) {
+  int v;
+  if (!g.sorted_ids) {
+    v = g.T - blk * BN;
+  } else {
+    const unsigned slots = static_cast<unsigned>(g.T * g.top_k);
+    int c = 0;
+    for (int i = lane; i < BN; i += 32) c += static_cast<unsigned>(g.sorted_ids[blk * BN + i]) < slots ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    v = c;
+  }
+  v = (v + 15) & ~15;
+  return v < 16 ? 16 : (v > BN ? BN : v);
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -387,7 +408,8 @@ __device__ void quantize_rows_grid(const GemmArgs& g, int rows) {
 
 template <int BN, int STAGES, bool S1, int KIND>
 __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
-    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
   using L = GemmSmem<BN, STAGES, KIND>;
   constexpr bool FP8 = KIND == kFp8;
   constexpr bool MX = KIND == kMx8;
@@ -395,7 +417,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
   constexpr int NACC = L::kAcc;
   constexpr int KE = KIND == kBf16 ? 64 : 128;  // K elements per stage
   constexpr int kUmmaKBytes = 32;               // K bytes per MMA: 16 bf16 or 32 e4m3
-  constexpr uint32_t kIdesc = FP8 ? idesc_e4m3(kTileM, BN) : idesc_bf16(kTileM, BN);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
   static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
@@ -454,6 +475,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
       const int blk = tile / g.n_mt;
       const int mt = tile - blk * g.n_mt;
       const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+      const int ncols = block_cols<BN>(g, blk, lane);  // token rows this tile loads and multiplies
       if (S1 && !g.b_tile) {
         for (int i = lane; i < BN; i += 32) {
           const int r = blk * BN + i;
@@ -475,16 +497,13 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         if (!ok) break;
         if (lane == 0) {
           pending &= ~(1u << stage);
-          uint32_t bytes = L::kABytes + L::kBBytes;
+          uint32_t bytes = L::kABytes + static_cast<uint32_t>(ncols) * kTileKBytes;
           if (MX) bytes += 2 * kSfTile;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          if (S1) {
-            tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
-            if (g.b_tile) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
-          } else {
-            tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
-            tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
-          }
+          if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+          else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
+          // token rows as one box when the tile is full (B from x, the sorted copy, or h)
+          if ((!S1 || g.b_tile) && ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
           if (MX) {
             const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
             bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
@@ -495,12 +514,17 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
         }
         __syncwarp();
+        // the other token-row loads, issued by the lanes of the warp (the
+        // barrier was armed above with the stage's full byte count)
         if (S1 && !g.b_tile) {
-          // token rows, four per gather, issued by the lanes of the warp (the
-          // barrier was armed above with the stage's full byte count)
-          for (int q = lane; q < BN / 4; q += 32)
+          // four rows per gather
+          for (int q = lane; q < ncols / 4; q += 32)
             tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
                         rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
+        } else if (ncols < BN) {
+          // a short tile: 16-row boxes
+          for (int q = lane; q < ncols / 16; q += 32)
+            tma_load_2d(b_dst + q * 16 * kTileKBytes, &tmB16, &full[stage], kb * KE, blk * BN + q * 16, pol_x);
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -523,6 +547,8 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
       const int acc = j % NACC;
       const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
+      const int ncols = block_cols<BN>(g, tile / g.n_mt, lane);
+      const uint32_t idesc = FP8 ? idesc_e4m3(kTileM, ncols) : idesc_bf16(kTileM, ncols);
       if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -555,11 +581,11 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
             if (MX) {
               // K block kk of the stage: byte kk of each scale column
               const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, BN, kk), tsfa | sel, tsfb | sel, accum);
+              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, ncols, kk), tsfa | sel, tsfb | sel, accum);
             } else if (FP8) {
-              umma_f8(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
+              umma_f8(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
             } else {
-              umma_f16(d_tmem, adesc + adv, bdesc + adv, kIdesc, accum);
+              umma_f16(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
             }
           }
           umma_commit(&empty[stage]);  // smem stage free once these MMAs (and copies) finish
@@ -599,6 +625,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
       const int acc = j % NACC;
       const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
       const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+      const int ncols = block_cols<BN>(g, blk, lane);  // accumulator columns the MMA wrote
 
       // per-column metadata, fetched while the accumulator is still being built
       for (int c = et; c < BN; c += kEpiThreads) {
@@ -631,12 +658,14 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         const int feat = mt * 64 + 16 * q + (lane & 15);
         const bool lo = lane < 16;
         float hv_keep[MX ? BN / 2 : 1];  // MXFP8: h of this thread's columns until the block scale is known
-#pragma unroll 1
+        // (MXFP8 unrolls the column loop so that hv_keep stays in registers)
+#pragma unroll(MX ? BN / 16 : 1)
         for (int c0 = 0; c0 < BN; c0 += 16) {
+          if (c0 < ncols) {
           float v[16];
           tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
           tmem_wait_ld();
-          if (c0 + 16 >= BN) {
+          if (c0 + 16 >= ncols) {
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
           }
@@ -669,6 +698,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
               if ((lane & 15) == 0) amax_part[q * BN + c] = m;
             }
           }
+          }
         }
         if (MX) {
           // One MX block = 32 features = lane quarters 2p and 2p+1 of the tile
@@ -680,6 +710,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           const size_t tile_base = (static_cast<size_t>(blk) * (g.I / 128) + kblk / 4) * kSfTile;
 #pragma unroll
           for (int i = 0; i < BN / 2; ++i) {
+            if (2 * i >= ncols) continue;
             const int c = 2 * i + (lo ? 0 : 1);
             const float amax = fmaxf(amax_part[q * BN + c], amax_part[(q ^ 1) * BN + c]);
             const int X = mx_exponent(amax);
@@ -692,7 +723,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         }
         if (FP8) {
           named_bar_sync(bar_id, kEpiThreads);
-          for (int c = et; c < BN; c += kEpiThreads) {
+          for (int c = et; c < ncols; c += kEpiThreads) {
             const float m = fmaxf(fmaxf(amax_part[c], amax_part[BN + c]),
                                   fmaxf(amax_part[2 * BN + c], amax_part[3 * BN + c]));
             g.h_amax[static_cast<size_t>(mt) * g.rows_cap + blk * BN + c] = m;
@@ -719,11 +750,11 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         const int n = mt * kTileM + 32 * q + lane;  // output feature
         const bool nvalid = n < g.H;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
           float v[16];
           tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
           tmem_wait_ld();
-          if (c0 + 16 >= BN) {
+          if (c0 + 16 >= ncols) {
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);
           }

@@ -101,8 +101,8 @@ constexpr int stages_for() {
 }
 
 template <int BN, bool S1, int KIND>
-moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
-                            cudaStream_t s) {
+moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb16,
+                            const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   constexpr int ST = stages_for<BN, KIND>();
   using L = moe::GemmSmem<BN, ST, KIND>;
   static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
@@ -118,37 +118,38 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
   if (grid < 1) grid = 1;
   if (g.quant_phase) {
     // every CTA resident at once (one per SM): the grid barrier's wait ends
-    void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<moe::GemmArgs*>(&g)};
+    void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<CUtensorMap*>(&tb16),
+                    const_cast<moe::GemmArgs*>(&g)};
     MOE_CK(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
                                        dim3(moe::EpiCfg<BN, KIND>::kThreads), args, L::kBytes, s));
   } else {
-    kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, g);
+    kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, tb16, g);
   }
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
 
 template <bool S1, int KIND>
-moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g, int max_tiles,
-                         cudaStream_t s) {
+moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb16,
+                         const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   switch (bm) {
-    case 16: return launch_gemm_bn<16, S1, KIND>(ta, tb, g, max_tiles, s);
-    case 32: return launch_gemm_bn<32, S1, KIND>(ta, tb, g, max_tiles, s);
-    case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, g, max_tiles, s);
-    case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, g, max_tiles, s);
+    case 16: return launch_gemm_bn<16, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
+    case 32: return launch_gemm_bn<32, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
+    case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
+    case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
     case 256:
-      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, g, max_tiles, s);
+      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
       break;
   }
   return MOE_ERR_INVALID_ARG;
 }
 
 template <bool S1>
-moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb, const moe::GemmArgs& g,
-                              int max_tiles, cudaStream_t s) {
-  if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, g, max_tiles, s);
-  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, g, max_tiles, s);
-  return launch_gemm<S1, moe::kBf16>(bm, ta, tb, g, max_tiles, s);
+moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
+                              const CUtensorMap& tb16, const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
+  if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, tb16, g, max_tiles, s);
+  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, tb16, g, max_tiles, s);
+  return launch_gemm<S1, moe::kBf16>(bm, ta, tb, tb16, g, max_tiles, s);
 }
 
 // Padded sorted length bound T*k + E*(bm-1), rounded up to whole blocks.
@@ -369,7 +370,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint8_t* xs = permute ? wsb + L.xs_off : nullptr;
   uint8_t* xsf = mx ? wsb + L.xsf_off : nullptr;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb16;
   {
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(H), 16, 2, static_cast<cuuint64_t>(I / 16),
                                 static_cast<cuuint64_t>(E)};
@@ -383,13 +384,21 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     // token rows: one [block_m x 128 B] box per stage from x (identity
     // routing; rows past T read as zeros) or from the sorted copy; else
     // single rows of x for tile::gather4
+    // (tb16: the same rows in 16-row boxes, for tiles with fewer token rows)
     const bool tile = permute || !sorted_ids;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), permute ? static_cast<cuuint64_t>(rows_cap)
                                                                     : static_cast<cuuint64_t>(T)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
+    const void* base = permute ? static_cast<const void*>(xs) : x;
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), tile ? static_cast<cuuint32_t>(block_m) : 1u};
-    moe_status_t r = make_map(&tb, tdt, 2, permute ? static_cast<const void*>(xs) : x, dims, st, box);
+    moe_status_t r = make_map(&tb, tdt, 2, base, dims, st, box);
     if (r != MOE_OK) return r;
+    tb16 = tb;
+    if (tile) {
+      const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
+      r = make_map(&tb16, tdt, 2, base, dims, st, box16);
+      if (r != MOE_OK) return r;
+    }
   }
   moe::GemmArgs g{};
   g.sorted_ids = sorted_ids;
@@ -447,7 +456,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     MOE_CK(cudaGetLastError());
   }
   const int max_tiles = cap_blocks * g.n_mt;
-  return launch_gemm_kind<true>(dtype, block_m, ta, tb, g, max_tiles, s);
+  return launch_gemm_kind<true>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
 moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_scale, const void* w2,
@@ -482,7 +491,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   // identity routing launches over the blocks that hold tokens only
   const int cap_blocks = sorted_ids ? static_cast<int>(rows_cap / block_m) : (T + block_m - 1) / block_m;
   const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb16;
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(E)};
@@ -496,6 +505,9 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(I) * es};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
     moe_status_t r = make_map(&tb, tdt, 2, h, dims, st, box);
+    if (r != MOE_OK) return r;
+    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
+    r = make_map(&tb16, tdt, 2, h, dims, st, box16);
     if (r != MOE_OK) return r;
   }
   cudaStream_t s = as_stream(stream);
@@ -528,7 +540,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
-  return launch_gemm_kind<false>(dtype, block_m, ta, tb, g, max_tiles, s);
+  return launch_gemm_kind<false>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
 size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I) {
