@@ -168,6 +168,46 @@ def _desc_order(keys: np.ndarray) -> np.ndarray:
     return np.argsort(-keys, axis=-1, kind="stable")
 
 
+ROUTER_CHUNKS = 8
+
+
+def router_logits(x, w_r, logit_bias=None, chunks: int = ROUTER_CHUNKS) -> np.ndarray:
+    """Router logits ``x . W_r`` in one fixed fp32 order (float32 result [T, E]).
+
+    The pages give no arithmetic for the router linear (vllm-project/vllm
+    PR 65207, "Purpose", passes the gating output to ``biased_grouped_topk``);
+    the fused router of this implementation defines one order, written out here
+    so that routing decisions made from these logits can be compared bit for
+    bit: with ``c = H / chunks``, for each chunk j the fp32 running sum
+    ``p_j = (...((x_{jc} w_{jc}) + x_{jc+1} w_{jc+1}) + ...)`` in index order,
+    then ``logit = (...((p_0 + p_1) + p_2) + ...) + p_{chunks-1}``, then
+    ``+ logit_bias[e]`` (fp32) when given. Every addition rounds to nearest
+    fp32. The products of bf16 or fp16 inputs are exact in fp32 (at most
+    8 + 8 or 11 + 11 significant bits), so only the additions round; this is
+    asserted for the inputs given.
+
+    x: [T, H] values of a bf16/fp16 tensor; w_r: [H, E] of the same format.
+    """
+    x = np.asarray(x, np.float64)
+    w = np.asarray(w_r, np.float64)
+    T, H = x.shape
+    H2, E = w.shape
+    assert H == H2 and H % chunks == 0
+    c = H // chunks
+    out = None
+    for j in range(chunks):
+        acc = np.zeros((T, E), np.float32)
+        for h in range(j * c, (j + 1) * c):
+            prod = np.outer(x[:, h], w[h, :])
+            p32 = prod.astype(np.float32)
+            assert np.array_equal(p32.astype(np.float64), prod), "product not exact in fp32"
+            acc = acc + p32
+        out = acc if out is None else out + acc
+    if logit_bias is not None:
+        out = out + np.asarray(logit_bias, np.float32)[None, :]
+    return out
+
+
 def router_softmax_topk(logits, top_k: int, renormalize: bool = True, rsf: float = 1.0):
     """Softmax top-k.
 

@@ -131,6 +131,57 @@ def _brute_topk(keys, k):
     raise AssertionError
 
 
+# ------------------------------------------------------------ router logits
+
+
+def test_router_logits_small_integers_equal_the_exact_matmul():
+    # integers |x|, |w| <= 8 over H = 64: every partial sum is an integer far
+    # below 2^24, so any order gives the exact product; a dropped, repeated or
+    # transposed term would not (T, H, E all different)
+    rng = np.random.default_rng(3)
+    x = rng.integers(-8, 9, (3, 64)).astype(np.float64)
+    w = rng.integers(-8, 9, (64, 5)).astype(np.float64)
+    got = oracle.router_logits(x, w)
+    assert got.dtype == np.float32 and got.shape == (3, 5)
+    assert np.array_equal(got.astype(np.float64), x @ w)
+    bias = np.array([0.5, -1.0, 2.0, 0.0, 3.25])
+    assert np.array_equal(oracle.router_logits(x, w, bias).astype(np.float64), x @ w + bias)
+
+
+def test_router_logits_chunk_order_hand_cases():
+    # H = 16, 8 chunks of 2. Row of ones against one expert column:
+    # w = [2^24, 0 | 1, 1 | 0 ...]: chunk sums 2^24 and 2 add exactly
+    # (2^24 + 2); one running sum over all 16 terms would stay at 2^24.
+    x = np.ones((1, 16))
+    w = np.zeros((16, 1))
+    w[0, 0], w[2, 0], w[3, 0] = 2.0**24, 1.0, 1.0
+    assert oracle.router_logits(x, w)[0, 0] == 2.0**24 + 2
+    # w = [2^24, 1 | 1, 0 ...]: chunk 0 rounds 2^24 + 1 to 2^24 (ties to
+    # even), then 2^24 + 1 rounds to 2^24 again: the exact sum is 2^24 + 2.
+    w[:] = 0
+    w[0, 0], w[1, 0], w[2, 0] = 2.0**24, 1.0, 1.0
+    assert oracle.router_logits(x, w)[0, 0] == 2.0**24
+    # the same three terms all inside chunk 1 round the same way
+    w[:] = 0
+    w[2, 0], w[3, 0] = 2.0**24, 1.0
+    w[4, 0] = 1.0
+    assert oracle.router_logits(x, w)[0, 0] == 2.0**24
+
+
+def test_router_logits_within_the_fp32_summation_bound():
+    # bf16 inputs: products exact, each of the H/8 - 1 + 7 additions on a
+    # path rounds by at most 2^-24 relative to its partial sum
+    g = torch.Generator().manual_seed(5)
+    T, H, E = 6, 2048, 40
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16).double().numpy()
+    w = (torch.randn(H, E, generator=g) * 0.02).to(torch.bfloat16).double().numpy()
+    got = oracle.router_logits(x, w).astype(np.float64)
+    exact = x @ w
+    bound = (H // 8 + 8) * 2.0**-24 * (np.abs(x) @ np.abs(w))
+    assert np.all(np.abs(got - exact) <= bound)
+    assert np.any(got != exact)  # the rounding is really fp32
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_softmax_topk_brute_force_with_ties(seed):
     rng = np.random.default_rng(seed)
