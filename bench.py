@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--unroll", type=int, default=20, help="steps per captured graph")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router-gemm", action="store_true",
+                    help="start each step from the router linear x . W_r (moe_router_gemm_topk) instead of logits")
     return ap.parse_args()
 
 
@@ -175,7 +177,7 @@ def barrier(world: int):
         dist.barrier()
 
 
-def algorithmic_bytes(cfg, counts):
+def algorithmic_bytes(cfg, counts, router_gemm=False):
     """Bytes the layer and each GEMM must move at minimum (weights of the
     experts the routing activates, activations in and out once)."""
     el = 2 if cfg.dtype == "bf16" else 1
@@ -190,6 +192,8 @@ def algorithmic_bytes(cfg, counts):
     s2 = active * w2 + h + out + out + rows * 4  # h in, out, addend in, top-k weights
     shared = synth.shared_weight_bytes(cfg)
     layer = active * (w13 + w2) + shared + x + out + cfg.T * cfg.E * 4 + (cfg.H * 2 if cfg.shared_gate else 0)
+    if router_gemm:  # W_r and the bf16 x it multiplies (the logits are then written, not read)
+        layer += cfg.H * cfg.E * 2 + (cfg.T * cfg.H * 2 if cfg.dtype != "bf16" else 0)
     return {"active_experts": active, "stage1": s1, "stage2": s2, "layer": layer}
 
 
@@ -211,7 +215,9 @@ def run_ours(args):
 
     cfg = configs.CONFIGS[args.config]
     inp = synth.make_layer_inputs(cfg, device=dev)
-    layer = MoELayer(cfg, inp)
+    if args.router_gemm and cfg.dtype == "bf16":
+        inp["x_r"] = inp["x"]  # the same bf16 activations feed the router linear and stage 1
+    layer = MoELayer(cfg, inp, router_gemm=args.router_gemm)
     main = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(main):
         layer.forward(main)
@@ -219,7 +225,7 @@ def run_ours(args):
     if capi.device_error(main) != 0:
         raise RuntimeError("device error after the first step")
     counts = layer.expert_counts.cpu()
-    ab = algorithmic_bytes(cfg, counts)
+    ab = algorithmic_bytes(cfg, counts, args.router_gemm)
 
     # graphs: U unrolled plain steps, the same U steps with timing events
     # around the two GEMMs (events inside a graph add a few microseconds each,
@@ -288,14 +294,16 @@ def run_ours(args):
 
     # e2e through the public API with host buffers: H2D of x and logits from
     # pinned memory, the five calls, D2H of the output, every step
-    x_h = inp["x"].cpu().pin_memory()
-    lg_h = inp["logits"].cpu().pin_memory()
+    # step inputs copied from pinned host memory: x, and either the logits or
+    # (fused router, quantised layers) the bf16 x of the router linear
+    names = ["x"] + ((["x_r"] if cfg.dtype != "bf16" else []) if args.router_gemm else ["logits"])
+    hosts = [inp[n].cpu().pin_memory() for n in names]
     out_h = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
     E2E = args.e2e_steps
     with torch.cuda.stream(main):
         for _ in range(3):
-            inp["x"].copy_(x_h, non_blocking=True)
-            inp["logits"].copy_(lg_h, non_blocking=True)
+            for n, hsrc in zip(names, hosts):
+                inp[n].copy_(hsrc, non_blocking=True)
             layer.forward(main)
             out_h.copy_(layer.out, non_blocking=True)
     torch.cuda.synchronize()
@@ -305,8 +313,8 @@ def run_ours(args):
     e0.record(main)
     with torch.cuda.stream(main):
         for _ in range(E2E):
-            inp["x"].copy_(x_h, non_blocking=True)
-            inp["logits"].copy_(lg_h, non_blocking=True)
+            for n, hsrc in zip(names, hosts):
+                inp[n].copy_(hsrc, non_blocking=True)
             layer.forward(main)
             out_h.copy_(layer.out, non_blocking=True)
     e1.record(main)
@@ -327,7 +335,8 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": cfg.dtype,
         "data": "synthetic",
-        "config": {"workload": workload_desc(cfg), "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T,
+        "config": {"workload": workload_desc(cfg) + (" +router_gemm" if args.router_gemm else ""),
+                   "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas{world}", "l2": "no flush: activated weights "
                    f"{ab['layer'] / 1e9:.2f} GB per step > 126 MB L2", "graph": f"CUDA graphs of {U} steps; the last {U} carry timing events",
                    "block_m": layer.bm, "active_experts": ab["active_experts"]},
@@ -339,7 +348,7 @@ def run_ours(args):
         "kernels_us": {"stage1": s1_us, "addend_wait": wait_us, "stage2": s2_us,
                        "note": "from the last U steps, whose graph carries timing events"},
         "e2e": {"value": tokens * E2E / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size(),
+                "h2d_bytes_per_step": sum(hs.numel() * hs.element_size() for hs in hosts),
                 "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": E2E,
                 "api": "MoELayer.forward (eager C-ABI calls)"},
         "gpu_launches": K * layer.launches_per_step,

@@ -171,6 +171,36 @@ moe_status_t moe_router_topk(const float* logits, const float* correction_bias, 
                              float routed_scaling_factor, int32_t* topk_ids, float* topk_weights,
                              moe_stream_t stream);
 
+/* moe_router_gemm_topk: the router linear and the top-k in one call:
+ *     logits = x . W_r (+ logit_bias), then moe_router_topk's selection.
+ * The pages give no arithmetic for the router linear ([65207] "Purpose" passes
+ * the gate linear's output to the top-k); this call defines one fixed fp32
+ * order so that its logits, and every decision taken from them, can be
+ * reproduced bit for bit on any machine:
+ *     c = H / 8; p_j = fp32 running sum of x[t,h] * W_r[h,e] over
+ *     h = j*c .. j*c + c - 1 in index order (j = 0..7);
+ *     logit = (...((p_0 + p_1) + p_2) + ...) + p_7, then + logit_bias[e].
+ * Every addition rounds to nearest fp32; products of bf16 or fp16 values are
+ * exact in fp32, so they do not round (products below the fp32 normal range,
+ * impossible for fp16 and absent for bf16 inputs of ordinary magnitude, would).
+ * One cluster of 8 CTAs per 4 tokens (16 once T >= 64 and E <= 256): CTA j
+ * sums chunk j, streaming its rows of W_r through shared memory by bulk copy,
+ * and writes its partial sums into CTA 0's shared memory (distributed shared
+ * memory); CTA 0 adds them in chunk order and selects.
+ *   dtype       MOE_DT_BF16 or MOE_DT_FP16: the type of x and W_r.
+ *   x           [T,H] row-major; W_r [H,E] row-major (E contiguous).
+ *   logit_bias  fp32 [E] or NULL, added to the logits before routing.
+ *   logits      fp32 [T,E] output or NULL: the logits the routing used.
+ *   other arguments, outputs and checks: as moe_router_topk, plus
+ *   H % 8 == 0 and E % 8 == 0 (MOE_ERR_SHAPE), W_r 16-byte aligned
+ *   (MOE_ERR_ALIGNMENT); MOE_ERR_SHAPE also if the shared-memory layout does
+ *   not fit one CTA (H = 7168 with E = 512 fits). */
+moe_status_t moe_router_gemm_topk(int dtype, const void* x, const void* w_r, const float* logit_bias,
+                                  const float* correction_bias, int T, int H, int E, int top_k,
+                                  int mode, int n_group, int topk_group, int renormalize,
+                                  float routed_scaling_factor, float* logits, int32_t* topk_ids,
+                                  float* topk_weights, moe_stream_t stream);
+
 /* moe_align_sort: group the T*k routed slots by expert for the grouped GEMMs
  * ([65207] reviewer measurements: moe_sorting; here it never zeroes the layer
  * output - the stage-2 epilogue owns the output; [6106]: the GEMM rows follow

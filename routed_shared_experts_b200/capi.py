@@ -35,6 +35,7 @@ SIGNATURES = {
     "moe_mx_h_scale_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_mx_pack_weight_scales": (_I, [_I, _P, _P, _I, _I, _I, _P]),
     "moe_router_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "moe_router_gemm_topk": (_I, [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "moe_align_sort": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_stage1_gemm": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_stage2_gemm_accumulate": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P,
@@ -136,6 +137,17 @@ def moe_router_topk(logits, correction_bias, top_k, mode, n_group, topk_group, r
     _check("moe_router_topk", lib().moe_router_topk(
         _ptr(logits), _ptr(correction_bias), T, E, top_k, mode, n_group, topk_group, int(renormalize),
         float(routed_scaling_factor), _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+
+
+def moe_router_gemm_topk(x, w_r, logit_bias, correction_bias, top_k, mode, n_group, topk_group, renormalize,
+                         routed_scaling_factor, logits, topk_ids, topk_weights, stream=None):
+    T, H = x.shape
+    E = w_r.shape[1]
+    dtype = MOE_DT_BF16 if x.dtype == torch.bfloat16 else MOE_DT_FP16
+    _check("moe_router_gemm_topk", lib().moe_router_gemm_topk(
+        dtype, _ptr(x), _ptr(w_r), _ptr(logit_bias), _ptr(correction_bias), T, H, E, top_k, mode, n_group,
+        topk_group, int(renormalize), float(routed_scaling_factor), _ptr(logits), _ptr(topk_ids),
+        _ptr(topk_weights), _stream(stream)))
 
 
 def moe_align_sort(topk_ids, E, block_m, sorted_ids, block_expert, expert_counts, expert_offsets, num_padded,

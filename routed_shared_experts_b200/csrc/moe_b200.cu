@@ -210,6 +210,61 @@ moe_status_t static_ws_address(void** out) {
 
 // ======================================================================== ABI
 
+// Argument checks shared by the two routing entry points.
+moe_status_t check_route(const float* correction_bias, int T, int E, int top_k, int mode, int n_group,
+                         int topk_group, const int32_t* topk_ids, const float* topk_weights) {
+  if (!topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOPK)
+    return MOE_ERR_INVALID_ARG;
+  if (mode != MOE_ROUTE_SOFTMAX && mode != MOE_ROUTE_GROUPED_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (mode == MOE_ROUTE_GROUPED_SIGMOID) {
+    if (n_group < 1 || n_group > 32 || E % n_group != 0) return MOE_ERR_INVALID_ARG;
+    if (topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
+    if (top_k > topk_group * (E / n_group)) return MOE_ERR_INVALID_ARG;
+  } else if (correction_bias) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+template <int VPL, int TB, typename TX>
+moe_status_t launch_router_gemm(moe::RouterGemmArgs a, cudaStream_t s) {
+  auto kern = moe::k_router_gemm_topk<VPL, TB, TX>;
+  const int c = a.H / moe::kRouterChunks;
+  // W_r ring: up to 4 buffers of up to 64 rows, at least two sub-chunks per
+  // chunk (both first buffers load at once); shrink the rows, then the number
+  // of buffers, until the layout fits 227 KB
+  int R = (c + 1) / 2 < 64 ? (c + 1) / 2 : 64;
+  int NB = moe::kRouterMaxBuf;
+  auto bytes = [&]() { return moe::RouterGemmSmem(TB, 32 * VPL, a.r.E, c, R, NB).total; };
+  while (bytes() > 227u * 1024 && (R > 8 || NB > 2)) {
+    if (NB > 2) --NB;
+    else R /= 2;
+  }
+  const size_t smem = bytes();
+  if (smem > 227u * 1024) return MOE_ERR_SHAPE;
+  a.rows_per_stage = R;
+  a.nbuf = NB;
+  MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  const dim3 grid(moe::kRouterChunks, (a.r.T + TB - 1) / TB);
+  kern<<<grid, moe::kRouterGemmThreads, smem, s>>>(a);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+template <typename TX>
+moe_status_t launch_router_gemm_vpl(const moe::RouterGemmArgs& a, cudaStream_t s) {
+  // 16 tokens per cluster once there are enough tokens to fill clusters of them
+  // (W_r is then read once per 16 tokens), 4 otherwise (more clusters at decode)
+  const int vpl = (a.r.E + 31) / 32;
+  const bool wide = a.r.T >= 64 && vpl <= 8;
+  if (vpl <= 1) return wide ? launch_router_gemm<1, 16, TX>(a, s) : launch_router_gemm<1, 4, TX>(a, s);
+  if (vpl <= 2) return wide ? launch_router_gemm<2, 16, TX>(a, s) : launch_router_gemm<2, 4, TX>(a, s);
+  if (vpl <= 4) return wide ? launch_router_gemm<4, 16, TX>(a, s) : launch_router_gemm<4, 4, TX>(a, s);
+  if (vpl <= 8) return wide ? launch_router_gemm<8, 16, TX>(a, s) : launch_router_gemm<8, 4, TX>(a, s);
+  return launch_router_gemm<16, 4, TX>(a, s);
+}
+
 extern "C" {
 
 const char* moe_status_string(moe_status_t s) {
@@ -260,20 +315,35 @@ size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int
   return Stage1Ws(dtype, capacity(T, top_k, E, block_m), H, I, block_m).total;
 }
 
+moe_status_t moe_router_gemm_topk(int dtype, const void* x, const void* w_r, const float* logit_bias,
+                                  const float* correction_bias, int T, int H, int E, int top_k, int mode, int n_group,
+                                  int topk_group, int renormalize, float routed_scaling_factor, float* logits,
+                                  int32_t* topk_ids, float* topk_weights, moe_stream_t stream) {
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!x || !w_r) return MOE_ERR_INVALID_ARG;
+  const moe_status_t r = check_route(correction_bias, T, E, top_k, mode, n_group, topk_group, topk_ids, topk_weights);
+  if (r != MOE_OK) return r;
+  if (H < moe::kRouterChunks || H % moe::kRouterChunks != 0 || E % 8 != 0) return MOE_ERR_SHAPE;
+  if (!aligned16(w_r)) return MOE_ERR_ALIGNMENT;  // W_r rows are bulk-copied
+  moe::RouterGemmArgs a{};
+  a.x = x;
+  a.w = w_r;
+  a.logit_bias = logit_bias;
+  a.H = H;
+  a.x_vec = (H % 64 == 0 && aligned16(x)) ? 1 : 0;
+  a.logits_out = logits;
+  a.r = moe::RouterArgs{nullptr, correction_bias, T, E, top_k, mode, n_group, topk_group, renormalize,
+                        routed_scaling_factor, topk_ids, topk_weights};
+  cudaStream_t s = as_stream(stream);
+  return dtype == MOE_DT_BF16 ? launch_router_gemm_vpl<__nv_bfloat16>(a, s) : launch_router_gemm_vpl<__half>(a, s);
+}
+
 moe_status_t moe_router_topk(const float* logits, const float* correction_bias, int T, int E, int top_k, int mode,
                              int n_group, int topk_group, int renormalize, float routed_scaling_factor,
                              int32_t* topk_ids, float* topk_weights, moe_stream_t stream) {
-  if (!logits || !topk_ids || !topk_weights) return MOE_ERR_INVALID_ARG;
-  if (T < 1 || E < 1 || E > MOE_MAX_EXPERTS || top_k < 1 || top_k > E || top_k > MOE_MAX_TOPK)
-    return MOE_ERR_INVALID_ARG;
-  if (mode != MOE_ROUTE_SOFTMAX && mode != MOE_ROUTE_GROUPED_SIGMOID) return MOE_ERR_INVALID_ARG;
-  if (mode == MOE_ROUTE_GROUPED_SIGMOID) {
-    if (n_group < 1 || n_group > 32 || E % n_group != 0) return MOE_ERR_INVALID_ARG;
-    if (topk_group < 1 || topk_group > n_group) return MOE_ERR_INVALID_ARG;
-    if (top_k > topk_group * (E / n_group)) return MOE_ERR_INVALID_ARG;
-  } else if (correction_bias) {
-    return MOE_ERR_INVALID_ARG;
-  }
+  if (!logits) return MOE_ERR_INVALID_ARG;
+  const moe_status_t r = check_route(correction_bias, T, E, top_k, mode, n_group, topk_group, topk_ids, topk_weights);
+  if (r != MOE_OK) return r;
   moe::RouterArgs a{logits, correction_bias, T, E, top_k, mode, n_group, topk_group, renormalize,
                     routed_scaling_factor, topk_ids, topk_weights};
   const int vpl = (E + 31) / 32;

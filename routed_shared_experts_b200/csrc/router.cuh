@@ -4,6 +4,8 @@
 // is applied to the top-k weights inside the top-k kernel (biased grouped
 // top-k), so no multiply of the layer output follows.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "ptx.cuh"
 
 namespace moe {
@@ -49,18 +51,13 @@ __device__ __forceinline__ float warp_max_f(float v) {
 
 constexpr int kRouterWarps = 4;
 
-// VPL = values per lane = ceil(E / 32). Expert e lives in lane e % 32, slot e / 32.
+// Top-k of token t from its logits row `l` (global or shared memory), run by
+// one warp. VPL = values per lane = ceil(E / 32): expert e lives in lane
+// e % 32, slot e / 32. c_sm / s_sm: E floats each of this warp's shared
+// scratch (grouped mode).
 template <int VPL>
-__global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(const RouterArgs a) {
-  extern __shared__ float rsm[];  // per warp: c[E], s[E] (grouped mode)
-  const int wib = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kRouterWarps + wib;
-  if (t >= a.T) return;
+__device__ void route_token(const RouterArgs& a, const float* l, float* c_sm, float* s_sm, int t, int lane) {
   const int E = a.E;
-  float* c_sm = rsm + wib * 2 * E;
-  float* s_sm = c_sm + E;
-  const float* l = a.logits + static_cast<size_t>(t) * E;
   const float NEG_INF = __int_as_float(0xff800000);
 
   float key[VPL];
@@ -178,6 +175,271 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(const RouterA
     a.ids[static_cast<size_t>(t) * a.k + lane] = my_sel;
     a.wts[static_cast<size_t>(t) * a.k + lane] = static_cast<float>(w);
   }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(const RouterArgs a) {
+  extern __shared__ float rsm[];  // per warp: c[E], s[E] (grouped mode)
+  const int wib = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRouterWarps + wib;
+  if (t >= a.T) return;
+  float* c_sm = rsm + wib * 2 * a.E;
+  route_token<VPL>(a, a.logits + static_cast<size_t>(t) * a.E, c_sm, c_sm + a.E, t, lane);
+}
+
+
+// ---------------------------------------------------------------------------
+// Fused router linear + top-k: logits = x . W_r in one fixed fp32 order, then
+// route_token. The pages give no router arithmetic (vllm-project/vllm
+// PR 65207, "Purpose", passes the gate linear's output to the top-k); the
+// order is this implementation's definition: H in kRouterChunks contiguous
+// chunks, each summed in index order in fp32, the chunk sums added in chunk
+// order, then the fp32 logit bias. Products of bf16/fp16 values are exact in
+// fp32, so fmaf(x, w, acc) rounds exactly like acc + (x * w).
+//
+// One cluster of kRouterChunks CTAs per TB tokens: CTA j of the cluster sums
+// chunk j for the cluster's tokens and all experts, streaming its rows of W_r
+// through a two-buffer shared-memory ring (one bulk copy per sub-chunk of
+// `rows_per_stage` rows), and writes the partial sums into CTA 0's shared
+// memory (distributed shared memory); after the cluster barrier CTA 0 adds
+// them in chunk order and its warps select the top-k of the TB tokens.
+
+constexpr int kRouterChunks = 8;
+constexpr int kRouterGemmThreads = 256;
+constexpr int kRouterMaxBuf = 4;  // deepest W_r ring
+
+struct RouterGemmArgs {
+  const void* x;            // [T, H], bf16 or fp16
+  const void* w;            // [H, E], same type (E % 8 == 0)
+  const float* logit_bias;  // [E] or nullptr
+  int H, rows_per_stage, nbuf;  // W_r ring: nbuf buffers of rows_per_stage rows
+  int x_vec;          // 1: x and H / 8 allow 16-byte loads of every chunk row
+  float* logits_out;  // [T, E] or nullptr
+  RouterArgs r;       // routing parameters and outputs (r.logits unused)
+};
+
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_float(__half v) { return __half2float(v); }
+template <typename TX>
+__device__ __forceinline__ TX bits_as(unsigned short b);
+template <>
+__device__ __forceinline__ __nv_bfloat16 bits_as<__nv_bfloat16>(unsigned short b) {
+  return __ushort_as_bfloat16(b);
+}
+template <>
+__device__ __forceinline__ __half bits_as<__half>(unsigned short b) {
+  return __ushort_as_half(b);
+}
+// The two values packed in a 32-bit word (low half first), without taking
+// the address of a register.
+__device__ __forceinline__ void unpack2(uint32_t w, __nv_bfloat16, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ void unpack2(uint32_t w, __half, float& lo, float& hi) {
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+
+// Shared-memory layout of k_router_gemm_topk (byte offsets; the W ring first,
+// 128-byte aligned, then the partial sums, the selection scratch, x and the
+// two ring barriers).
+struct RouterGemmSmem {
+  size_t w_off, part_off, cs_off, xs_off, bar_off, total;
+  __host__ __device__ RouterGemmSmem(int TB, int EP, int E, int chunk, int rows, int nbuf) {
+    auto up = [](size_t v) { return (v + 127) / 128 * 128; };
+    w_off = 0;
+    part_off = up(static_cast<size_t>(nbuf) * rows * E * 2);
+    cs_off = part_off + up(static_cast<size_t>(kRouterChunks) * TB * EP * 4);
+    xs_off = cs_off + up(static_cast<size_t>(kRouterGemmThreads / 32) * 2 * E * 4);
+    bar_off = xs_off + up(static_cast<size_t>(chunk) * TB * 2);
+    total = bar_off + 8 * kRouterMaxBuf;
+  }
+};
+
+template <int VPL, int TB, typename TX>
+__global__ void __cluster_dims__(kRouterChunks, 1, 1) __launch_bounds__(kRouterGemmThreads)
+    k_router_gemm_topk(const RouterGemmArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int j = static_cast<int>(cluster.block_rank());
+  const int E = a.r.E;
+  const int H = a.H;
+  const int c = H / kRouterChunks;
+  const int R = a.rows_per_stage;
+  const int NB = a.nbuf;
+  const int nsub = (c + R - 1) / R;
+  const int t0 = blockIdx.y * TB;
+  const int tid = threadIdx.x;
+  constexpr int EP = 32 * VPL;  // experts padded to whole lanes
+  extern __shared__ __align__(128) uint8_t rg_raw[];
+  const RouterGemmSmem L(TB, EP, E, c, R, NB);
+  TX* wbuf = reinterpret_cast<TX*>(rg_raw + L.w_off);       // [NB][R][E]
+  float* part = reinterpret_cast<float*>(rg_raw + L.part_off);  // [chunk][token][EP], CTA 0
+  float* cs = reinterpret_cast<float*>(rg_raw + L.cs_off);      // per warp: c[E], s[E], CTA 0
+  TX* xs = reinterpret_cast<TX*>(rg_raw + L.xs_off);            // [h][token]: x of chunk j, transposed
+  uint64_t* bar = reinterpret_cast<uint64_t*>(rg_raw + L.bar_off);
+  __shared__ int abort_sm;
+  const TX* x = static_cast<const TX*>(a.x);
+  const TX* wj = static_cast<const TX*>(a.w) + static_cast<size_t>(j) * c * E;
+
+  auto issue = [&](int sub) {  // thread 0: rows [sub*R, sub*R + rows) of chunk j into buffer sub % NB
+    const int rows = min(R, c - sub * R);
+    const uint32_t bytes = static_cast<uint32_t>(rows) * E * 2;
+    const int b = sub % NB;
+    mbar_arrive_expect_tx(&bar[b], bytes);
+    bulk_load(wbuf + b * R * E, wj + static_cast<size_t>(sub) * R * E, bytes, &bar[b], policy_evict_last());
+  };
+  if (tid == 0) {
+    abort_sm = 0;
+    for (int b = 0; b < NB; ++b) mbar_init(&bar[b], 1);
+    fence_barrier_init();
+    for (int sub = 0; sub < NB && sub < nsub; ++sub) issue(sub);
+  }
+  // x of chunk j for the cluster's tokens, transposed to [h][token]: 16-byte
+  // loads (8 values) when every row segment is 16-byte aligned, all issued
+  // before any is stored
+  if (a.x_vec) {
+    const int per_tok = c / 8;
+    constexpr int kMaxV = 8;
+    for (int base = tid; base < TB * per_tok; base += kRouterGemmThreads * kMaxV) {
+      uint4 v[kMaxV];
+#pragma unroll
+      for (int u = 0; u < kMaxV; ++u) {
+        const int i = base + u * kRouterGemmThreads;
+        const int tt = i / per_tok;
+        const int t = t0 + tt;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (i < TB * per_tok && t < a.r.T)
+          v[u] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + j * c) + (i - tt * per_tok));
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxV; ++u) {
+        const int i = base + u * kRouterGemmThreads;
+        if (i < TB * per_tok) {
+          const int tt = i / per_tok;
+          const int h0 = (i - tt * per_tok) * 8;
+          const uint32_t wv4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            xs[(h0 + 2 * q) * TB + tt] = bits_as<TX>(static_cast<unsigned short>(wv4[q] & 0xffffu));
+            xs[(h0 + 2 * q + 1) * TB + tt] = bits_as<TX>(static_cast<unsigned short>(wv4[q] >> 16));
+          }
+        }
+      }
+    }
+  } else {
+    for (int i = tid; i < TB * c; i += kRouterGemmThreads) {
+      const int tt = i / c;
+      const int h = i - tt * c;
+      const int t = t0 + tt;
+      xs[h * TB + tt] = t < a.r.T ? x[static_cast<size_t>(t) * H + j * c + h] : TX(0.0f);
+    }
+  }
+  __syncthreads();
+
+  // Thread mapping: NE experts e_lo + k*EPT and TPT consecutive tokens
+  // grp*TPT + u per thread; a warp shares its tokens (broadcast reads of x).
+  constexpr int NE = EP > kRouterGemmThreads ? EP / kRouterGemmThreads : 1;
+  constexpr int EPT = EP / NE;
+  constexpr int G = kRouterGemmThreads / EPT;
+  constexpr int TPT = TB >= G ? TB / G : 1;
+  const int e_lo = tid % EPT;
+  const int grp = tid / EPT;
+  const bool has_tok = grp * TPT < TB;
+  float acc[TPT][NE];
+#pragma unroll
+  for (int u = 0; u < TPT; ++u)
+#pragma unroll
+    for (int k = 0; k < NE; ++k) acc[u][k] = 0.f;
+  bool live = true;
+  for (int sub = 0; sub < nsub; ++sub) {
+    if (live && !mbar_wait(&bar[sub % NB], static_cast<uint32_t>(sub / NB) & 1u, &abort_sm)) live = false;
+    if (live && has_tok) {
+      const TX* wb = wbuf + (sub % NB) * R * E;
+      const TX* xr = xs + static_cast<size_t>(sub) * R * TB + grp * TPT;
+      const int rows = min(R, c - sub * R);
+#pragma unroll 4
+      for (int i = 0; i < rows; ++i) {
+        float xv[TPT];
+        if constexpr (TPT % 8 == 0) {
+#pragma unroll
+          for (int v = 0; v < TPT / 8; ++v) {
+            const uint4 q = *reinterpret_cast<const uint4*>(xr + i * TB + 8 * v);
+            unpack2(q.x, TX(), xv[8 * v + 0], xv[8 * v + 1]);
+            unpack2(q.y, TX(), xv[8 * v + 2], xv[8 * v + 3]);
+            unpack2(q.z, TX(), xv[8 * v + 4], xv[8 * v + 5]);
+            unpack2(q.w, TX(), xv[8 * v + 6], xv[8 * v + 7]);
+          }
+        } else if constexpr (TPT == 4) {
+          const uint2 q = *reinterpret_cast<const uint2*>(xr + i * TB);
+          unpack2(q.x, TX(), xv[0], xv[1]);
+          unpack2(q.y, TX(), xv[2], xv[3]);
+        } else if constexpr (TPT == 2) {
+          unpack2(*reinterpret_cast<const uint32_t*>(xr + i * TB), TX(), xv[0], xv[1]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < TPT; ++u) xv[u] = to_float(xr[i * TB + u]);
+        }
+        float wv[NE];
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+          const int e = e_lo + k * EPT;
+          wv[k] = e < E ? to_float(wb[i * E + e]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < TPT; ++u)
+#pragma unroll
+          for (int k = 0; k < NE; ++k) acc[u][k] = fmaf(xv[u], wv[k], acc[u][k]);
+      }
+    }
+    __syncthreads();  // buffer sub % NB is no longer read
+    if (tid == 0 && live && !abort_sm && sub + NB < nsub) issue(sub + NB);
+  }
+  if (tid == 0 && abort_sm) {
+    // a wait gave up: let the copies still in flight land (bounded) before leaving
+    for (int sub = 0; sub < nsub && sub < NB; ++sub) {
+      const uint64_t t_start = globaltimer();
+      while (!mbar_try_wait(smem_u32(&bar[sub % NB]), static_cast<uint32_t>(sub / NB) & 1u) &&
+             globaltimer() - t_start < kWaitTimeoutNs) {
+      }
+    }
+  }
+
+  float* part0 = cluster.map_shared_rank(part, 0);
+  if (has_tok) {
+#pragma unroll
+    for (int u = 0; u < TPT; ++u)
+#pragma unroll
+      for (int k = 0; k < NE; ++k) {
+        const int e = e_lo + k * EPT;
+        if (e < E) part0[(j * TB + grp * TPT + u) * EP + e] = acc[u][k];
+      }
+  }
+  cluster.sync();
+  if (j != 0) return;
+
+  // chunk sums in chunk order (+ logit bias), written back into chunk 0's slot
+  for (int q = tid; q < TB * EP; q += kRouterGemmThreads) {
+    const int tt = q / EP;
+    const int e = q - tt * EP;
+    if (e >= E) continue;
+    float v = part[tt * EP + e];
+#pragma unroll
+    for (int k = 1; k < kRouterChunks; ++k) v = __fadd_rn(v, part[(k * TB + tt) * EP + e]);
+    if (a.logit_bias) v = __fadd_rn(v, a.logit_bias[e]);
+    part[tt * EP + e] = v;
+    const int t = t0 + tt;
+    if (a.logits_out && t < a.r.T) a.logits_out[static_cast<size_t>(t) * E + e] = v;
+  }
+  __syncthreads();
+  const int wib = tid >> 5;
+  const int lane = tid & 31;
+  float* c_sm = cs + wib * 2 * E;
+  for (int tt = wib; tt < TB; tt += kRouterGemmThreads / 32)
+    if (t0 + tt < a.r.T) route_token<VPL>(a.r, part + tt * EP, c_sm, c_sm + E, t0 + tt, lane);
 }
 
 }  // namespace moe

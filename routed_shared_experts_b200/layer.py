@@ -24,11 +24,16 @@ class MoELayer:
     ``inp`` is a dict from ``synth.make_layer_inputs`` (tensors already on the
     device). Weights are referenced, not copied; activations (``x``,
     ``logits``) are read from the same dict at every forward, so a caller may
-    refill them in place.
+    refill them in place. With ``router_gemm`` the step starts from the router
+    linear instead of the logits: ``moe_router_gemm_topk`` on ``x_r`` (bf16),
+    ``w_r`` [H,E] and ``logit_bias``, writing the logits it used to
+    ``self.logits``.
     """
 
-    def __init__(self, cfg: MoEConfig, inp: dict, block_m: int | None = None, device=None):
+    def __init__(self, cfg: MoEConfig, inp: dict, block_m: int | None = None, device=None,
+                 router_gemm: bool = False):
         self.cfg = cfg
+        self.router_gemm = router_gemm
         self.inp = inp
         self.device = torch.device(device or inp["x"].device)
         dev = self.device
@@ -42,6 +47,7 @@ class MoELayer:
         i32 = dict(dtype=torch.int32, device=dev)
         self.topk_ids = torch.empty((T, k), **i32)
         self.topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=dev) if router_gemm else None
         self.sorted_ids = torch.empty(cap, **i32)
         self.block_expert = torch.empty(cap // bm, **i32)
         self.expert_counts = torch.empty(E, **i32)
@@ -105,8 +111,13 @@ class MoELayer:
         cfg, inp = self.cfg, self.inp
         T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I
         mode = capi.MOE_ROUTE_SOFTMAX if cfg.route == "softmax" else capi.MOE_ROUTE_GROUPED_SIGMOID
-        capi.moe_router_topk(inp["logits"], inp.get("correction_bias"), k, mode, cfg.n_group, cfg.topk_group,
-                             cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, stream)
+        if self.router_gemm:
+            capi.moe_router_gemm_topk(inp["x_r"], inp["w_r"], inp["logit_bias"], inp.get("correction_bias"), k,
+                                      mode, cfg.n_group, cfg.topk_group, cfg.renormalize, cfg.rsf, self.logits,
+                                      self.topk_ids, self.topk_weights, stream)
+        else:
+            capi.moe_router_topk(inp["logits"], inp.get("correction_bias"), k, mode, cfg.n_group, cfg.topk_group,
+                                 cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, stream)
         capi.moe_align_sort(self.topk_ids, E, self.bm, self.sorted_ids, self.block_expert, self.expert_counts,
                             self.expert_offsets, self.num_padded, stream)
         if probes:

@@ -18,7 +18,9 @@ Input formats (the layer's inputs arrive already in their storage format):
 
 Router logits are the model's gate linear, which lies before the layer: they are
 made here as fp32 ``x @ W_r`` (from the unrounded draws) plus a per-expert logit
-bias, and handed to both sides as the same fp32 tensor.
+bias, and handed to both sides as the same fp32 tensor. For the fused router
+path the same draws are also returned in bf16: ``x_r`` (x), ``w_r`` (W_r, [H,E])
+and the fp32 ``logit_bias``.
 """
 from __future__ import annotations
 
@@ -100,7 +102,8 @@ def make_layer_inputs(cfg: MoEConfig, device="cpu") -> dict:
     logits = (x32 @ w_r + lbias[None, :]).float().contiguous()
     w_gate32 = _randn((H,), g, device, std) if cfg.shared_gate else None
 
-    inp = {"logits": logits}
+    inp = {"logits": logits, "x_r": x32.to(torch.bfloat16), "w_r": w_r.to(torch.bfloat16).contiguous(),
+           "logit_bias": lbias.float().contiguous()}
     # x: per-token scale (fp8) -> one scale per row
     inp["x"], inp["x_scale"] = _store(x32, fmt, 1)
     del x32

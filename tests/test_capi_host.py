@@ -94,6 +94,23 @@ def test_router_rejects(lib):
 
 
 @no_gpu
+def test_router_gemm_rejects(lib):
+    f = lib.moe_router_gemm_topk
+
+    def call(dt=capi.MOE_DT_BF16, x=P, w=P, T=4, H=256, E=8, k=2, mode=0, cb=None):
+        return f(dt, x, w, None, cb, T, H, E, k, mode, 1, 1, 1, 1.0, None, P, P, None)
+    assert call(dt=capi.MOE_DT_F32) == -2
+    assert call(dt=capi.MOE_DT_FP8_E4M3) == -2
+    assert call(x=None) == -1
+    assert call(w=None) == -1
+    assert call(H=252) == -4                        # H % 8
+    assert call(E=12) == -4                         # E % 8 (W_r rows are bulk-copied)
+    assert call(w=P + 8) == -3
+    assert call(k=9) == -1
+    assert call(cb=P) == -1                         # correction bias only in grouped mode
+
+
+@no_gpu
 def test_sort_rejects(lib):
     f = lib.moe_align_sort
     assert f(None, 4, 2, 8, 16, P, P, P, P, P, None) == -1
