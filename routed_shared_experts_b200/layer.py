@@ -152,4 +152,11 @@ class MoELayer:
     # kernels this library launches per forward()
     @property
     def launches_per_step(self) -> int:
-        return 6 + (1 if self.gate is not None else 0)
+        """Kernels this library launches per forward()."""
+        cfg = self.cfg
+        route = 2  # top-k (or router linear + top-k), then the sort
+        mx = cfg.dtype == "mxfp8"
+        prep_routed = 1 if (mx or self.bm >= 32) else 0  # sorted token copy / token scale tiles
+        prep_shared = 1 if mx else 0
+        gate = 1 if self.gate is not None else 0
+        return route + prep_routed + 2 + gate + prep_shared + 2
