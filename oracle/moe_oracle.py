@@ -155,6 +155,51 @@ def mx_block_exponent(amax) -> np.ndarray:
     return np.where(a == 0, -127, x)
 
 
+def e4m3_encode(values) -> np.ndarray:
+    """Codes (uint8) of values that are already e4m3 numbers (finite, |v| <= 448):
+    the inverse of e4m3_decode, with +0 for zero."""
+    v = np.asarray(values, np.float64)
+    finite = ~np.isnan(E4M3_TABLE)
+    codes = np.nonzero(finite)[0]
+    order = np.argsort(E4M3_TABLE[finite], kind="stable")
+    table_v = E4M3_TABLE[finite][order]
+    table_c = codes[order]
+    idx = np.searchsorted(table_v, v)
+    idx = np.clip(idx, 0, len(table_v) - 1)
+    assert np.array_equal(table_v[idx], v), "not an e4m3 value"
+    out = table_c[idx].astype(np.uint8)
+    return np.where(v == 0, np.uint8(0), out)  # -0 and +0 both encode as +0
+
+
+def quantize_activations(x, mode: str):
+    """Quantisation of the layer's bf16 activations x [T, H] to the stage-1
+    operand formats (ROCm/aiter PR 6106, "Technical Details": per-token
+    activation scales; MXFP8 with BLOCK_K = 32). Returns (codes uint8 [T, H],
+    scales): fp32 [T] for 'fp8', ue8m0 bytes [T, H/32] for 'mxfp8'.
+
+    'fp8': s = fp32(amax / 448) per row (amax = 0 gives s = 1); each code is
+    e4m3_rn(fp32(x / s)) with saturation - the quotient rounded to fp32 first,
+    the precision the kernel decides in, then to e4m3.
+    'mxfp8': per 32 columns X = mx_block_exponent(amax), byte X + 127, codes
+    e4m3_rn(x * 2^-X) (exact scaling, then one rounding).
+    """
+    x = np.asarray(x, np.float64)
+    T, H = x.shape
+    if mode == "fp8":
+        amax = np.max(np.abs(x), axis=1)
+        s = np.where(amax > 0, fp32_round(amax / E4M3_MAX), 1.0)
+        q = fp32_round(x.astype(np.float32) / s.astype(np.float32)[:, None])
+        vals = round_to_format(q, E4M3)
+        return e4m3_encode(vals), s.astype(np.float32)
+    if mode == "mxfp8":
+        assert H % 32 == 0
+        blk = x.reshape(T, H // 32, 32)
+        X = mx_block_exponent(np.max(np.abs(blk), axis=-1))
+        vals = round_to_format(blk * np.ldexp(1.0, -X.astype(np.int32))[..., None], E4M3)
+        return e4m3_encode(vals.reshape(T, H)), (X + 127).astype(np.uint8)
+    raise ValueError(mode)
+
+
 # ---------------------------------------------------------------------------
 # Router (top-k). vllm PR 65207, "Purpose", commit 1: routed_scaling_factor is
 # folded into the top-k weights inside the top-k kernel.

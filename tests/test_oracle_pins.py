@@ -131,6 +131,48 @@ def _brute_topk(keys, k):
     raise AssertionError
 
 
+# ------------------------------------------------------ activation quantisation
+
+
+def test_e4m3_encode_inverts_decode():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF, 0x80)])
+    assert np.array_equal(oracle.e4m3_encode(mo.e4m3_decode(codes)), codes)
+    assert oracle.e4m3_encode(np.array([-0.0]))[0] == 0
+
+
+def test_quantize_activations_fp8_matches_torch_division_and_cast():
+    # torch: fp32 division by the fp32 scale, float8_e4m3fn cast (RNE); an
+    # independent implementation of the same two roundings
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(8, 512, generator=g).to(torch.bfloat16)
+    x[3] = 0
+    x[5, 7] = 40.0  # one large element: the row's amax
+    codes, s = oracle.quantize_activations(x.double().numpy(), "fp8")
+    xf = x.float()
+    amax = xf.abs().amax(dim=1)
+    st = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    ref = (xf / st[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+    assert np.array_equal(s, st.numpy())
+    assert np.all(codes[3] == 0) and s[3] == 1.0
+    assert codes[5, 7] == 0x7E  # the amax element maps to 448
+
+
+def test_quantize_activations_mx_matches_generator_rule_and_invariants():
+    g = torch.Generator().manual_seed(10)
+    x = torch.randn(4, 256, generator=g).to(torch.bfloat16)
+    x[1, 32:64] = 0  # an all-zero block
+    codes, sb = oracle.quantize_activations(x.double().numpy(), "mxfp8")
+    from routed_shared_experts_b200 import synth
+    rc, rs = synth.quant_mx(x.float())
+    assert np.array_equal(codes, rc.numpy()) and np.array_equal(sb, rs.numpy())
+    assert sb[1, 1] == 0 and np.all(codes[1, 32:64] == 0)
+    # every block's largest |code| value times 2^X stays within the block amax's e4m3 step
+    vals = mo.e4m3_decode(codes).reshape(4, 8, 32) * np.ldexp(1.0, sb.astype(np.int32) - 127)[..., None]
+    amax = np.abs(x.double().numpy()).reshape(4, 8, 32).max(-1)
+    assert np.all(np.abs(vals).max(-1) <= amax * (1 + 2.0**-3) + 1e-30)
+
+
 # ------------------------------------------------------------ router logits
 
 
