@@ -157,18 +157,15 @@ def mx_block_exponent(amax) -> np.ndarray:
 
 def e4m3_encode(values) -> np.ndarray:
     """Codes (uint8) of values that are already e4m3 numbers (finite, |v| <= 448):
-    the inverse of e4m3_decode, with +0 for zero."""
+    the inverse of e4m3_decode. E4M3 is sign-magnitude, so the sign bit comes
+    from the value's sign, zero included: a negative value that rounded to zero
+    (-0.0) encodes as 0x80, as the OCP format defines -0."""
     v = np.asarray(values, np.float64)
-    finite = ~np.isnan(E4M3_TABLE)
-    codes = np.nonzero(finite)[0]
-    order = np.argsort(E4M3_TABLE[finite], kind="stable")
-    table_v = E4M3_TABLE[finite][order]
-    table_c = codes[order]
-    idx = np.searchsorted(table_v, v)
-    idx = np.clip(idx, 0, len(table_v) - 1)
-    assert np.array_equal(table_v[idx], v), "not an e4m3 value"
-    out = table_c[idx].astype(np.uint8)
-    return np.where(v == 0, np.uint8(0), out)  # -0 and +0 both encode as +0
+    mag = np.abs(v)
+    table_v = E4M3_TABLE[:0x7F]  # codes 0x00..0x7E: the non-negative values, increasing
+    idx = np.clip(np.searchsorted(table_v, mag), 0, 0x7E)
+    assert np.array_equal(table_v[idx], mag), "not an e4m3 value"
+    return (idx | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
 
 
 def quantize_activations(x, mode: str):

@@ -135,9 +135,19 @@ def _brute_topk(keys, k):
 
 
 def test_e4m3_encode_inverts_decode():
-    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF, 0x80)])
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)])
     assert np.array_equal(oracle.e4m3_encode(mo.e4m3_decode(codes)), codes)
-    assert oracle.e4m3_encode(np.array([-0.0]))[0] == 0
+    assert oracle.e4m3_encode(np.array([-0.0]))[0] == 0x80 and oracle.e4m3_encode(np.array([0.0]))[0] == 0
+
+
+def test_quantize_activations_keeps_the_sign_of_zero_like_torch():
+    # a large outlier makes s large, so tiny values round to +-0: negative ones
+    # encode as 0x80 in torch's float8_e4m3fn cast as in the oracle
+    x = torch.tensor([[300.0, -1e-4, 1e-4, -0.0, 0.0, -3e-4, 5.0, -5.0]]).to(torch.bfloat16)
+    codes, s = oracle.quantize_activations(x.double().numpy(), "fp8")
+    ref = (x.float() / torch.tensor(s)[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+    assert codes[0, 1] == 0x80 and codes[0, 2] == 0x00
 
 
 def test_quantize_activations_fp8_matches_torch_division_and_cast():
