@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-gemm", action="store_true",
                     help="start each step from the router linear x . W_r (moe_router_gemm_topk) instead of logits")
+    ap.add_argument("--quantize-x", action="store_true",
+                    help="fp8/MXFP8 layers: start each step from bf16 x (moe_quantize_activations)")
     return ap.parse_args()
 
 
@@ -177,7 +179,7 @@ def barrier(world: int):
         dist.barrier()
 
 
-def algorithmic_bytes(cfg, counts, router_gemm=False):
+def algorithmic_bytes(cfg, counts, router_gemm=False, quantize_x=False):
     """Bytes the layer and each GEMM must move at minimum (weights of the
     experts the routing activates, activations in and out once)."""
     el = 2 if cfg.dtype == "bf16" else 1
@@ -192,8 +194,15 @@ def algorithmic_bytes(cfg, counts, router_gemm=False):
     s2 = active * w2 + h + out + out + rows * 4  # h in, out, addend in, top-k weights
     shared = synth.shared_weight_bytes(cfg)
     layer = active * (w13 + w2) + shared + x + out + cfg.T * cfg.E * 4 + (cfg.H * 2 if cfg.shared_gate else 0)
+    bf16_x_read = False
     if router_gemm:  # W_r and the bf16 x it multiplies (the logits are then written, not read)
-        layer += cfg.H * cfg.E * 2 + (cfg.T * cfg.H * 2 if cfg.dtype != "bf16" else 0)
+        layer += cfg.H * cfg.E * 2
+        bf16_x_read = cfg.dtype != "bf16"
+    if quantize_x:  # bf16 x read, its codes written (then read as before)
+        layer += cfg.T * cfg.H
+        bf16_x_read = True
+    if bf16_x_read:
+        layer += cfg.T * cfg.H * 2
     return {"active_experts": active, "stage1": s1, "stage2": s2, "layer": layer}
 
 
@@ -217,7 +226,7 @@ def run_ours(args):
     inp = synth.make_layer_inputs(cfg, device=dev)
     if args.router_gemm and cfg.dtype == "bf16":
         inp["x_r"] = inp["x"]  # the same bf16 activations feed the router linear and stage 1
-    layer = MoELayer(cfg, inp, router_gemm=args.router_gemm)
+    layer = MoELayer(cfg, inp, router_gemm=args.router_gemm, quantize_x=args.quantize_x)
     main = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(main):
         layer.forward(main)
@@ -225,7 +234,7 @@ def run_ours(args):
     if capi.device_error(main) != 0:
         raise RuntimeError("device error after the first step")
     counts = layer.expert_counts.cpu()
-    ab = algorithmic_bytes(cfg, counts, args.router_gemm)
+    ab = algorithmic_bytes(cfg, counts, args.router_gemm, args.quantize_x)
 
     # graphs: U unrolled plain steps, the same U steps with timing events
     # around the two GEMMs (events inside a graph add a few microseconds each,
@@ -294,9 +303,16 @@ def run_ours(args):
 
     # e2e through the public API with host buffers: H2D of x and logits from
     # pinned memory, the five calls, D2H of the output, every step
-    # step inputs copied from pinned host memory: x, and either the logits or
-    # (fused router, quantised layers) the bf16 x of the router linear
-    names = ["x"] + ((["x_r"] if cfg.dtype != "bf16" else []) if args.router_gemm else ["logits"])
+    # step inputs copied from pinned host memory: the activations the step
+    # reads (bf16 x when the step quantises it, else x in the layer's format),
+    # and the logits unless the step starts from the router linear, which
+    # reads bf16 x (the same tensor for a bf16 layer or with --quantize-x)
+    names = ["x_r" if args.quantize_x else "x"]
+    if args.router_gemm:
+        if cfg.dtype != "bf16" and not args.quantize_x:
+            names.append("x_r")
+    else:
+        names.append("logits")
     hosts = [inp[n].cpu().pin_memory() for n in names]
     out_h = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
     E2E = args.e2e_steps
@@ -335,7 +351,8 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": cfg.dtype,
         "data": "synthetic",
-        "config": {"workload": workload_desc(cfg) + (" +router_gemm" if args.router_gemm else ""),
+        "config": {"workload": workload_desc(cfg) + (" +router_gemm" if args.router_gemm else "")
+                   + (" +quantize_x" if args.quantize_x else ""),
                    "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas{world}", "l2": "no flush: activated weights "
                    f"{ab['layer'] / 1e9:.2f} GB per step > 126 MB L2", "graph": f"CUDA graphs of {U} steps; the last {U} carry timing events",

@@ -219,6 +219,21 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
                             int32_t* sorted_ids, int32_t* block_expert, int32_t* expert_counts,
                             int32_t* expert_offsets, int32_t* num_padded, moe_stream_t stream);
 
+/* moe_quantize_activations: the layer's bf16 activations x [T,H] to the
+ * stage-1 operand formats, so that bf16 x can enter an fp8 or MXFP8 layer
+ * ([6106] "Technical Details": per-token activation scales; BLOCK_K = 32).
+ *   dtype MOE_DT_FP8_E4M3: scale fp32 [T], s = amax(x_t)/448 (1 for an
+ *         all-zero row); codes [T,H] = e4m3(x / s), the quotient an IEEE fp32
+ *         division, round to nearest even, saturating to +-448.
+ *   dtype MOE_DT_MXFP8_E4M3: scale = ue8m0 bytes [T, H/32], X + 127 with
+ *         X = floor(log2 amax) - 8 per 32 columns (clamped to [-127,127],
+ *         -127 for an all-zero block); codes e4m3(x * 2^-X).
+ * One CTA per token row. Checks: H % 8 == 0 (fp8) / % 32 == 0 (MXFP8),
+ * H <= 16384, x 16-byte aligned, codes 8-byte aligned. Asynchronous on
+ * `stream`. */
+moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, void* codes, void* scale,
+                                      moe_stream_t stream);
+
 /* moe_stage1_gemm: per sorted row r (slot f = sorted_ids[r], token t = f/k,
  * expert e = block_expert[r/block_m]):
  *     a   = W13[e] . x[t]                           (2I outputs, fp32 accumulate)

@@ -43,6 +43,7 @@ SIGNATURES = {
     "moe_stage2_gemm_accumulate_static_ws": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                                   _P, _P, _P, _P]),
     "shared_expert_gate_dot": (_I, [_I, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_quantize_activations": (_I, [_I, _P, _I, _I, _P, _P, _P]),
 }
 
 _LIB = None
@@ -183,6 +184,12 @@ def moe_stage2_gemm_accumulate_static_ws(dtype, h, h_scale, w2, w2_scale, weight
         dtype, _ptr(h), _ptr(h_scale), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
         _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
         _event(addend_ready), _ptr(out), _stream(stream)))
+
+
+def moe_quantize_activations(dtype, x, codes, scale, stream=None):
+    T, H = x.shape
+    _check("moe_quantize_activations", lib().moe_quantize_activations(
+        dtype, _ptr(x), T, H, _ptr(codes), _ptr(scale), _stream(stream)))
 
 
 def shared_expert_gate_dot(dtype, x, w, apply_sigmoid, out, stream=None):

@@ -383,6 +383,22 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
   return MOE_OK;
 }
 
+moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, void* codes, void* scale,
+                                      moe_stream_t stream) {
+  const bool mx = dtype == MOE_DT_MXFP8_E4M3;
+  if (dtype != MOE_DT_FP8_E4M3 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!x || !codes || !scale || T < 1 || H < 1) return MOE_ERR_INVALID_ARG;
+  if (H % (mx ? 32 : 8) != 0 || H > moe::kQuantXThreads * 8 * moe::kQuantXMaxV) return MOE_ERR_SHAPE;
+  if (!aligned16(x) || reinterpret_cast<uintptr_t>(codes) % 8 != 0) return MOE_ERR_ALIGNMENT;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* q = static_cast<uint8_t*>(codes);
+  cudaStream_t s = as_stream(stream);
+  if (mx) moe::k_quantize_x<true><<<T, moe::kQuantXThreads, 0, s>>>(xb, H, q, nullptr, static_cast<uint8_t*>(scale));
+  else moe::k_quantize_x<false><<<T, moe::kQuantXThreads, 0, s>>>(xb, H, q, static_cast<float*>(scale), nullptr);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
 moe_status_t shared_expert_gate_dot(int dtype, const void* x, const void* w, int T, int K, int apply_sigmoid,
                                     void* out, moe_stream_t stream) {
   if (!x || !w || !out || T < 1 || K < 1) return MOE_ERR_INVALID_ARG;

@@ -27,13 +27,19 @@ class MoELayer:
     refill them in place. With ``router_gemm`` the step starts from the router
     linear instead of the logits: ``moe_router_gemm_topk`` on ``x_r`` (bf16),
     ``w_r`` [H,E] and ``logit_bias``, writing the logits it used to
-    ``self.logits``.
+    ``self.logits``. With ``quantize_x`` (fp8 / MXFP8 layers) the step starts
+    from the bf16 activations ``x_r``: ``moe_quantize_activations`` writes
+    ``self.xq`` / ``self.xq_scale``, which both GEMM paths then read instead
+    of ``x`` / ``x_scale``.
     """
 
     def __init__(self, cfg: MoEConfig, inp: dict, block_m: int | None = None, device=None,
-                 router_gemm: bool = False):
+                 router_gemm: bool = False, quantize_x: bool = False):
         self.cfg = cfg
         self.router_gemm = router_gemm
+        if quantize_x and cfg.dtype == "bf16":
+            raise ValueError("quantize_x applies to the fp8 and MXFP8 layers")
+        self.quantize_x = quantize_x
         self.inp = inp
         self.device = torch.device(device or inp["x"].device)
         dev = self.device
@@ -48,6 +54,11 @@ class MoELayer:
         self.topk_ids = torch.empty((T, k), **i32)
         self.topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
         self.logits = torch.empty((T, E), dtype=torch.float32, device=dev) if router_gemm else None
+        self.xq = self.xq_scale = None
+        if quantize_x:
+            self.xq = torch.empty((T, H), dtype=torch.uint8, device=dev)
+            self.xq_scale = (torch.empty(T, dtype=torch.float32, device=dev) if cfg.dtype == "fp8"
+                             else torch.empty((T, H // 32), dtype=torch.uint8, device=dev))
         self.sorted_ids = torch.empty(cap, **i32)
         self.block_expert = torch.empty(cap // bm, **i32)
         self.expert_counts = torch.empty(E, **i32)
@@ -88,22 +99,29 @@ class MoELayer:
         self.side = torch.cuda.Stream(device=dev)
         self.ev_in = torch.cuda.Event()
         self.ev_addend = torch.cuda.Event()
+        self.ev_q = torch.cuda.Event()
 
     # -- the two halves -------------------------------------------------------
+
+    def _x(self):
+        """Stage-1 activations and their scales."""
+        if self.quantize_x:
+            return self.xq, self.xq_scale
+        return self.inp["x"], self.inp.get("x_scale")
 
     def shared_expert(self, stream):
         cfg, inp = self.cfg, self.inp
         T, H, Is = cfg.T, cfg.H, cfg.Is
         if self.gate is not None:
             capi.shared_expert_gate_dot(capi.MOE_DT_BF16, inp["x"], inp["w_gate"], True, self.gate, stream)
-        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13s"], self.wsc["w13s"],
+        capi.moe_stage1_gemm(self.dt, *self._x(), inp["w13s"], self.wsc["w13s"],
                              None, None, None, T, 1, H, Is, 1, self.bm, self.h_s, self.h_scale_s, self.ws1_s, stream)
         wdt = capi.MOE_DT_BF16 if self.gate is not None else capi.MOE_DT_F32
         capi.moe_stage2_gemm_accumulate(self.dt, self.h_s, self.h_scale_s, inp["w2s"], self.wsc["w2s"],
                                         self.gate, wdt, None, None, None, T, 1, H, Is, 1, self.bm, None, None,
                                         None, self.addend, stream)
 
-    def routed(self, stream, addend=True, probes=None):
+    def routed(self, stream, addend=True, probes=None, wait_x=None):
         """Main-stream half. ``probes`` = optional four events recorded on
         ``stream``: before stage 1, after stage 1, before stage 2 (after its
         wait on the addend) and after stage 2. (Each recorded event costs a few
@@ -120,9 +138,11 @@ class MoELayer:
                                  cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, stream)
         capi.moe_align_sort(self.topk_ids, E, self.bm, self.sorted_ids, self.block_expert, self.expert_counts,
                             self.expert_offsets, self.num_padded, stream)
+        if wait_x is not None:  # the quantised activations (forward with quantize_x)
+            stream.wait_event(wait_x)
         if probes:
             probes[0].record(stream)
-        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), inp["w13"], self.wsc["w13"],
+        capi.moe_stage1_gemm(self.dt, *self._x(), inp["w13"], self.wsc["w13"],
                              self.sorted_ids, self.block_expert, self.num_padded, T, k, H, I, E, self.bm, self.h,
                              self.h_scale, self.ws1, stream)
         if probes:
@@ -144,9 +164,14 @@ class MoELayer:
         main = stream or torch.cuda.current_stream(self.device)
         self.ev_in.record(main)
         self.side.wait_event(self.ev_in)
+        if self.quantize_x:
+            # on the side stream, whose stage 1 needs the codes first; the main
+            # stream routes and sorts meanwhile and waits only before its stage 1
+            capi.moe_quantize_activations(self.dt, self.inp["x_r"], self.xq, self.xq_scale, self.side)
+            self.ev_q.record(self.side)
         self.shared_expert(self.side)
         self.ev_addend.record(self.side)
-        self.routed(main, probes=probes)
+        self.routed(main, probes=probes, wait_x=self.ev_q if self.quantize_x else None)
         return self.out
 
     # kernels this library launches per forward()
@@ -154,7 +179,7 @@ class MoELayer:
     def launches_per_step(self) -> int:
         """Kernels this library launches per forward()."""
         cfg = self.cfg
-        route = 2  # top-k (or router linear + top-k), then the sort
+        route = 2 + (1 if self.quantize_x else 0)  # (x quantisation,) top-k, sort
         mx = cfg.dtype == "mxfp8"
         prep_routed = 1 if (mx or self.bm >= 32) else 0  # sorted token copy / token scale tiles
         prep_shared = 1 if mx else 0

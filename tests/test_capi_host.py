@@ -111,6 +111,17 @@ def test_router_gemm_rejects(lib):
 
 
 @no_gpu
+def test_quantize_activations_rejects(lib):
+    f = lib.moe_quantize_activations
+    assert f(capi.MOE_DT_BF16, P, 4, 256, P, P, None) == -2
+    assert f(capi.MOE_DT_FP8_E4M3, None, 4, 256, P, P, None) == -1
+    assert f(capi.MOE_DT_FP8_E4M3, P, 0, 256, P, P, None) == -1
+    assert f(capi.MOE_DT_FP8_E4M3, P, 4, 252, P, P, None) == -4     # H % 8
+    assert f(capi.MOE_DT_MXFP8_E4M3, P, 4, 80, P, P, None) == -4    # H % 32
+    assert f(capi.MOE_DT_FP8_E4M3, P + 8, 4, 256, P, P, None) == -3
+
+
+@no_gpu
 def test_sort_rejects(lib):
     f = lib.moe_align_sort
     assert f(None, 4, 2, 8, 16, P, P, P, P, P, None) == -1
