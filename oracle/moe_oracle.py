@@ -545,7 +545,13 @@ def route(cfg, logits, correction_bias=None):
     )
 
 
-def moe_layer(cfg: dict, inp: dict, tokens=None) -> dict:
+def shared_pieces(Is: int, I: int) -> int:
+    """Number m of I-wide virtual experts that hold a shared expert of
+    intermediate size Is (the last one zero-padded)."""
+    return -(-Is // I)
+
+
+def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> dict:
     """Forward pass of one routed + shared-expert MoE layer, token by token.
 
     For each token t (all of them, or the listed ``tokens``):
@@ -564,6 +570,15 @@ def moe_layer(cfg: dict, inp: dict, tokens=None) -> dict:
     x_scale [T], w13_scale [E], w2_scale [E], w13s_scale [1], w2s_scale [1];
     mxfp8 configs add x_scale [T,H/32], w13_scale [E,2I,H/32], w2_scale
     [E,H,I/32], w13s_scale [2Is,H/32], w2s_scale [H,Is/32] (ue8m0 bytes).
+
+    ``shared_fused``: the shared expert taken as always-selected routed experts
+    (vllm-project/vllm PR 61503 "Fused heterogeneous MoE", "Overview"): it is cut
+    into m = ceil(Is / I) virtual experts of I intermediate features (gate rows
+    v*I..v*I+I-1 with their up rows and W2 columns, zero-padded past Is), each
+    computed like a routed expert (its h quantised on its own I columns) with
+    weight g_t, and all contributions meet before the one rounding:
+        out_t = bf16( sum_j w_j * Expert_{ids_j}(x_t) + sum_v g_t * Piece_v(x_t) )
+    ``addend`` then holds the unrounded shared sum.
 
     Returns routing for all tokens (ids, weights), and for the computed tokens:
     gate [n], addend [n,H], out [n,H] (float64 values of bf16 numbers) and
@@ -598,13 +613,28 @@ def moe_layer(cfg: dict, inp: dict, tokens=None) -> dict:
             return decode_operand(wt, fmt), float(s[0] if e is None else s[e])
         return decode_operand(wt, fmt), 1.0
 
-    # shared expert -> addend
+    # shared expert -> addend (or, fused, its unrounded sum over the pieces)
     w13s, s13s = weights_of("w13s")
     w2s, s2s = weights_of("w2s")
     addend = np.empty((len(tokens), H))
-    for i, t in enumerate(tokens):
-        ys = expert_forward(x_all[t], w13s, w2s, Is, fmt, s_x[t], s13s, s2s)
-        addend[i] = bf16_round(g[i] * ys)
+    if shared_fused:
+        m = shared_pieces(Is, I)
+        pieces = []
+        for v in range(m):
+            lo, hi = v * I, min((v + 1) * I, Is)
+            p13 = np.zeros((2 * I, H))
+            p13[: hi - lo] = w13s[lo:hi]
+            p13[I: I + hi - lo] = w13s[Is + lo: Is + hi]
+            p2 = np.zeros((H, I))
+            p2[:, : hi - lo] = w2s[:, lo:hi]
+            pieces.append((p13, p2))
+        for i, t in enumerate(tokens):
+            addend[i] = sum(g[i] * expert_forward(x_all[t], p13, p2, I, fmt, s_x[t], s13s, s2s)
+                            for p13, p2 in pieces)
+    else:
+        for i, t in enumerate(tokens):
+            ys = expert_forward(x_all[t], w13s, w2s, Is, fmt, s_x[t], s13s, s2s)
+            addend[i] = bf16_round(g[i] * ys)
 
     # routed experts: each (token, slot) pair is an independent expert call;
     # pairs are visited expert by expert only so that each expert's weights are

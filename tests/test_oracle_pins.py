@@ -508,6 +508,49 @@ def test_layer_equal_logits_give_uniform_weights():
     np.testing.assert_allclose(r["topk_weights"], 0.25, rtol=0)
 
 
+def test_shared_fused_equals_the_addend_path_up_to_the_addend_rounding():
+    # bf16 (h rounds per element, so cutting the shared expert into pieces does
+    # not change any h value): fused out = bf16(routed + g*S), addend path out =
+    # bf16(routed + bf16(g*S)); they differ only by the addend's rounding, and
+    # the fused shared sum equals the addend before its rounding
+    for Is in (128, 96, 320):  # Is = I, Is < I (one padded piece), Is > I (three pieces, the last padded)
+        cfg = _tiny_cfg(I=128, Is=Is)
+        inp = _tiny_inputs(cfg)
+        a = mo.moe_layer(cfg, inp)
+        f = mo.moe_layer(cfg, inp, shared_fused=True)
+        assert np.array_equal(a["addend"], mo.bf16_round(f["addend"]))
+        assert np.array_equal(f["out"], mo.bf16_round(f["routed"] + f["addend"]))
+        # one bf16 step of the output plus the addend's rounding (a bf16 step of
+        # |v| is at most |v| * 2^-7)
+        ulp = (np.maximum(np.abs(a["out"]), np.abs(f["out"])) + np.abs(a["addend"])) * 2.0**-7
+        assert np.all(np.abs(a["out"] - f["out"]) <= ulp + 1e-30)
+        assert np.mean(a["out"] == f["out"]) > 0.5
+    assert mo.shared_pieces(320, 128) == 3 and mo.shared_pieces(128, 128) == 1 and mo.shared_pieces(96, 128) == 1
+
+
+def test_shared_fused_fp8_pieces_take_their_own_row_scales():
+    # fp8: each piece's h row is quantised on its own I columns: with Is = 2I the
+    # fused shared output equals the sum of two half-size experts, each run
+    # through expert_forward on its own slice
+    cfg = dict(_tiny_cfg(I=128, Is=256), dtype="fp8", shared_gate=False)
+    g = np.random.default_rng(4)
+    E, H, I, Is, T = cfg["E"], cfg["H"], cfg["I"], cfg["Is"], cfg["T"]
+    codes = lambda *sh: g.integers(0, 0x7E, sh).astype(np.uint8) | (g.integers(0, 2, sh) * 0x80).astype(np.uint8)  # noqa: E731
+    inp = {"logits": g.normal(size=(T, E)).astype(np.float32), "x": codes(T, H), "x_scale": np.full(T, 0.01),
+           "w13": codes(E, 2 * I, H), "w2": codes(E, H, I), "w13_scale": np.full(E, 1e-3),
+           "w2_scale": np.full(E, 1e-3), "w13s": codes(2 * Is, H), "w2s": codes(H, Is),
+           "w13s_scale": np.array([2e-3]), "w2s_scale": np.array([5e-4])}
+    f = mo.moe_layer(cfg, inp, shared_fused=True, tokens=[0, 3])
+    x = mo.e4m3_decode(inp["x"])
+    w13s, w2s = mo.e4m3_decode(inp["w13s"]), mo.e4m3_decode(inp["w2s"])
+    for i, t in enumerate([0, 3]):
+        want = 0.0
+        for v in range(2):
+            p13 = np.concatenate([w13s[v * I:(v + 1) * I], w13s[Is + v * I: Is + (v + 1) * I]])
+            want = want + mo.expert_forward(x[t], p13, w2s[:, v * I:(v + 1) * I], I, "fp8", 0.01, 2e-3, 5e-4)
+        assert np.allclose(f["addend"][i], want, rtol=0, atol=1e-12)
+
+
 def test_layer_single_expert_is_dense_mlp():
     """E = 1, k = 1: the routed part is one dense MLP (checked with torch
     matmuls in float64 on the decoded weights)."""
