@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-gemm", action="store_true",
                     help="start each step from the router linear x . W_r (moe_router_gemm_topk) instead of logits")
+    ap.add_argument("--fused-shared", action="store_true",
+                    help="the shared expert as always-selected routed experts, one stream (FusedSharedMoELayer)")
     ap.add_argument("--quantize-x", action="store_true",
                     help="fp8/MXFP8 layers: start each step from bf16 x (moe_quantize_activations)")
     return ap.parse_args()
@@ -220,20 +222,25 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     from routed_shared_experts_b200 import capi
-    from routed_shared_experts_b200.layer import MoELayer
+    from routed_shared_experts_b200.layer import FusedSharedMoELayer, MoELayer
 
     cfg = configs.CONFIGS[args.config]
     inp = synth.make_layer_inputs(cfg, device=dev)
     if args.router_gemm and cfg.dtype == "bf16":
         inp["x_r"] = inp["x"]  # the same bf16 activations feed the router linear and stage 1
-    layer = MoELayer(cfg, inp, router_gemm=args.router_gemm, quantize_x=args.quantize_x)
+    if args.fused_shared:
+        if args.router_gemm or args.quantize_x:
+            raise SystemExit("--fused-shared runs from logits and pre-quantised x")
+        layer = FusedSharedMoELayer(cfg, inp)
+    else:
+        layer = MoELayer(cfg, inp, router_gemm=args.router_gemm, quantize_x=args.quantize_x)
     main = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(main):
         layer.forward(main)
     torch.cuda.synchronize()
     if capi.device_error(main) != 0:
         raise RuntimeError("device error after the first step")
-    counts = layer.expert_counts.cpu()
+    counts = layer.expert_counts.cpu()[: cfg.E]  # routed experts (the fused layer appends the shared pieces)
     ab = algorithmic_bytes(cfg, counts, args.router_gemm, args.quantize_x)
 
     # graphs: U unrolled plain steps, the same U steps with timing events
@@ -352,7 +359,7 @@ def run_ours(args):
         "dtype": cfg.dtype,
         "data": "synthetic",
         "config": {"workload": workload_desc(cfg) + (" +router_gemm" if args.router_gemm else "")
-                   + (" +quantize_x" if args.quantize_x else ""),
+                   + (" +quantize_x" if args.quantize_x else "") + (" +fused_shared" if args.fused_shared else ""),
                    "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas{world}", "l2": "no flush: activated weights "
                    f"{ab['layer'] / 1e9:.2f} GB per step > 126 MB L2", "graph": f"CUDA graphs of {U} steps; the last {U} carry timing events",

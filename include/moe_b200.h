@@ -219,6 +219,22 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
                             int32_t* sorted_ids, int32_t* block_expert, int32_t* expert_counts,
                             int32_t* expert_offsets, int32_t* num_padded, moe_stream_t stream);
 
+/* moe_append_shared_slots: the shared expert as always-selected routed
+ * experts ([61503] "Fused heterogeneous MoE", "Overview"). When the caller
+ * has appended the shared expert to the routed weights as m virtual experts
+ * E..E+m-1 (I intermediate features each, the last zero-padded past Is), this
+ * call extends every token's top-k by those m slots:
+ *   out_ids[t, 0..k-1] = topk_ids[t, :], out_ids[t, k+v] = E + v;
+ *   out_weights likewise, the appended slots weighted by gate[t] (bf16 or
+ *   fp16 per gate_dtype) or 1 when gate is NULL.
+ * moe_align_sort (E + m experts, k + m slots) and the two grouped GEMMs then
+ * compute routed and shared experts in the same launches, and stage 2 sums
+ * all k + m contributions before its one rounding (no addend, no side
+ * stream). Checks: E + m <= MOE_MAX_EXPERTS, k + m <= MOE_MAX_TOPK. */
+moe_status_t moe_append_shared_slots(const int32_t* topk_ids, const float* topk_weights, int T, int top_k,
+                                     int E, int m, const void* gate, int gate_dtype, int32_t* out_ids,
+                                     float* out_weights, moe_stream_t stream);
+
 /* moe_quantize_activations: the layer's bf16 activations x [T,H] to the
  * stage-1 operand formats, so that bf16 x can enter an fp8 or MXFP8 layer
  * ([6106] "Technical Details": per-token activation scales; BLOCK_K = 32).

@@ -44,6 +44,7 @@ SIGNATURES = {
                                                   _P, _P, _P, _P]),
     "shared_expert_gate_dot": (_I, [_I, _P, _P, _I, _I, _I, _P, _P]),
     "moe_quantize_activations": (_I, [_I, _P, _I, _I, _P, _P, _P]),
+    "moe_append_shared_slots": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
 }
 
 _LIB = None
@@ -184,6 +185,14 @@ def moe_stage2_gemm_accumulate_static_ws(dtype, h, h_scale, w2, w2_scale, weight
         dtype, _ptr(h), _ptr(h_scale), _ptr(w2), _ptr(w2_scale), _ptr(weights), weights_dtype,
         _ptr(sorted_ids), _ptr(block_expert), _ptr(num_padded), T, top_k, H, I, E, block_m, _ptr(addend),
         _event(addend_ready), _ptr(out), _stream(stream)))
+
+
+def moe_append_shared_slots(topk_ids, topk_weights, E, m, gate, out_ids, out_weights, stream=None):
+    T, k = topk_ids.shape
+    gdt = MOE_DT_FP16 if (gate is not None and gate.dtype == torch.float16) else MOE_DT_BF16
+    _check("moe_append_shared_slots", lib().moe_append_shared_slots(
+        _ptr(topk_ids), _ptr(topk_weights), T, k, E, m, _ptr(gate), gdt, _ptr(out_ids), _ptr(out_weights),
+        _stream(stream)))
 
 
 def moe_quantize_activations(dtype, x, codes, scale, stream=None):

@@ -383,6 +383,20 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
   return MOE_OK;
 }
 
+moe_status_t moe_append_shared_slots(const int32_t* topk_ids, const float* topk_weights, int T, int top_k, int E,
+                                     int m, const void* gate, int gate_dtype, int32_t* out_ids, float* out_weights,
+                                     moe_stream_t stream) {
+  if (!topk_ids || !topk_weights || !out_ids || !out_weights) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || m < 1 || E + m > MOE_MAX_EXPERTS || top_k + m > MOE_MAX_TOPK)
+    return MOE_ERR_INVALID_ARG;
+  if (gate && gate_dtype != MOE_DT_BF16 && gate_dtype != MOE_DT_FP16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const int n = T * (top_k + m);
+  moe::k_append_shared_slots<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(
+      topk_ids, topk_weights, T, top_k, E, m, gate, gate_dtype == MOE_DT_FP16 ? 1 : 0, out_ids, out_weights);
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
 moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, void* codes, void* scale,
                                       moe_stream_t stream) {
   const bool mx = dtype == MOE_DT_MXFP8_E4M3;

@@ -442,4 +442,28 @@ __global__ void __cluster_dims__(kRouterChunks, 1, 1) __launch_bounds__(kRouterG
     if (t0 + tt < a.r.T) route_token<VPL>(a.r, part + tt * EP, c_sm, c_sm + E, t0 + tt, lane);
 }
 
+// Fused shared expert (vllm-project/vllm PR 61503 "Fused heterogeneous MoE",
+// "Overview"): the shared expert held as m always-selected routed experts
+// E..E+m-1. Row t of the output top-k is the routed row followed by those m
+// slots, each weighted by the shared gate g_t (1 without a gate).
+__global__ void k_append_shared_slots(const int32_t* __restrict__ ids, const float* __restrict__ w, int T, int k,
+                                      int E, int m, const void* __restrict__ gate, int gate_half,
+                                      int32_t* __restrict__ ids2, float* __restrict__ w2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int km = k + m;
+  if (i >= T * km) return;
+  const int t = i / km;
+  const int j = i - t * km;
+  if (j < k) {
+    ids2[i] = ids[static_cast<size_t>(t) * k + j];
+    w2[i] = w[static_cast<size_t>(t) * k + j];
+  } else {
+    ids2[i] = E + (j - k);
+    float g = 1.0f;
+    if (gate) g = gate_half ? __half2float(static_cast<const __half*>(gate)[t])
+                            : __bfloat162float(static_cast<const __nv_bfloat16*>(gate)[t]);
+    w2[i] = g;
+  }
+}
+
 }  // namespace moe

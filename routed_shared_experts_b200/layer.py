@@ -185,3 +185,125 @@ class MoELayer:
         prep_shared = 1 if mx else 0
         gate = 1 if self.gate is not None else 0
         return route + prep_routed + 2 + gate + prep_shared + 2
+
+
+class FusedSharedMoELayer:
+    """The layer with the shared expert held as m = ceil(Is / I) always-selected
+    routed experts (vllm-project/vllm PR 61503 "Fused heterogeneous MoE",
+    "Overview"), on one stream:
+
+        [gate] -> top-k -> append the m shared slots (weight g_t or 1)
+               -> sort over E + m experts -> stage 1 -> stage 2 (k + m slots)
+
+    The shared weights are appended to the routed ones once, at construction:
+    virtual expert E + v holds intermediate features v*I .. v*I + I - 1 of the
+    shared expert (its gate rows, its up rows and its W2 columns), the last one
+    zero-padded past Is, with the shared expert's weight scales. All k + m
+    contributions meet in stage 2's fp32 workspace before the one bf16
+    rounding: no addend, no side stream, no event. Same interface as MoELayer
+    (``forward``, ``out``, ``topk_ids``, ``topk_weights``).
+    """
+
+    def __init__(self, cfg: MoEConfig, inp: dict, block_m: int | None = None, device=None):
+        self.cfg = cfg
+        self.inp = inp
+        self.device = torch.device(device or inp["x"].device)
+        dev = self.device
+        T, H, E, k, I, Is = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I, cfg.Is
+        self.m = m = -(-Is // I)
+        self.E2, self.k2 = E + m, k + m
+        self.bm = bm = block_m or cfg.block_m
+        self.dt = capi.DTYPES[cfg.dtype]
+        fp8 = cfg.dtype == "fp8"
+        mx = cfg.dtype == "mxfp8"
+
+        # combined weights [E + m, ...]: routed experts, then the shared pieces
+        w13s, w2s = inp["w13s"], inp["w2s"]
+        p13 = torch.zeros((m, 2 * I, H), dtype=w13s.dtype, device=dev)
+        p2 = torch.zeros((m, H, I), dtype=w2s.dtype, device=dev)
+        for v in range(m):
+            lo, hi = v * I, min((v + 1) * I, Is)
+            p13[v, : hi - lo] = w13s[lo:hi]
+            p13[v, I: I + hi - lo] = w13s[Is + lo: Is + hi]
+            p2[v, :, : hi - lo] = w2s[:, lo:hi]
+        self.w13 = torch.cat([inp["w13"], p13]).contiguous()
+        self.w2 = torch.cat([inp["w2"], p2]).contiguous()
+        self.wsc = {"w13": None, "w2": None}
+        if fp8:  # one fp32 scale per expert and matrix: the pieces take the shared one
+            self.wsc["w13"] = torch.cat([inp["w13_scale"].reshape(-1), inp["w13s_scale"].reshape(-1).repeat(m)])
+            self.wsc["w2"] = torch.cat([inp["w2_scale"].reshape(-1), inp["w2s_scale"].reshape(-1).repeat(m)])
+        elif mx:  # ue8m0 rows of the pieces (127 = 1.0 on the zero padding), then the tile layout
+            s13, s2 = inp["w13s_scale"], inp["w2s_scale"]
+            q13 = torch.full((m, 2 * I, H // 32), 127, dtype=torch.uint8, device=dev)
+            q2 = torch.full((m, H, I // 32), 127, dtype=torch.uint8, device=dev)
+            for v in range(m):
+                lo, hi = v * I, min((v + 1) * I, Is)
+                q13[v, : hi - lo] = s13[lo:hi]
+                q13[v, I: I + hi - lo] = s13[Is + lo: Is + hi]
+                q2[v, :, : (hi - lo) // 32] = s2[:, lo // 32: hi // 32]
+            for name, which, rows in (("w13", 0, torch.cat([inp["w13_scale"], q13])),
+                                      ("w2", 1, torch.cat([inp["w2_scale"], q2]))):
+                dst = torch.empty(capi.mx_weight_scale_bytes(which, self.E2, H, I), dtype=torch.uint8, device=dev)
+                capi.moe_mx_pack_weight_scales(which, rows.contiguous(), dst, self.E2, H, I)
+                self.wsc[name] = dst
+
+        cap = capi.sorted_capacity(T, self.k2, self.E2, bm)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.topk_ids = torch.empty((T, k), **i32)
+        self.topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.ids2 = torch.empty((T, self.k2), **i32)
+        self.w2slots = torch.empty((T, self.k2), dtype=torch.float32, device=dev)
+        self.sorted_ids = torch.empty(cap, **i32)
+        self.block_expert = torch.empty(cap // bm, **i32)
+        self.expert_counts = torch.empty(self.E2, **i32)
+        self.expert_offsets = torch.empty(self.E2 + 1, **i32)
+        self.num_padded = torch.empty(1, **i32)
+        hdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.uint8
+        self.h = torch.empty((cap, I), dtype=hdt, device=dev)
+        self.h_scale = None
+        if fp8:
+            self.h_scale = torch.empty(cap, dtype=torch.float32, device=dev)
+        elif mx:
+            self.h_scale = torch.zeros(capi.mx_h_scale_bytes(T, self.k2, self.E2, I, bm), dtype=torch.uint8,
+                                       device=dev)
+        ws1 = capi.stage1_workspace_bytes(self.dt, T, self.k2, self.E2, H, I, bm)
+        self.ws1 = torch.zeros(ws1, dtype=torch.uint8, device=dev) if ws1 else None  # zeroed once
+        self.gate = torch.empty(T, dtype=torch.bfloat16, device=dev) if cfg.shared_gate else None
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.acc_ws = torch.zeros(capi.stage2_workspace_bytes(T, H) // 4, dtype=torch.float32, device=dev)
+
+    def forward(self, stream=None, probes=None):
+        """Enqueue one layer step on ``stream``; returns ``self.out``. ``probes``:
+        optional four events around stage 1 and stage 2."""
+        cfg, inp = self.cfg, self.inp
+        T, H, E, k, I = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I
+        s = stream or torch.cuda.current_stream(self.device)
+        mode = capi.MOE_ROUTE_SOFTMAX if cfg.route == "softmax" else capi.MOE_ROUTE_GROUPED_SIGMOID
+        if self.gate is not None:
+            capi.shared_expert_gate_dot(capi.MOE_DT_BF16, inp["x"], inp["w_gate"], True, self.gate, s)
+        capi.moe_router_topk(inp["logits"], inp.get("correction_bias"), k, mode, cfg.n_group, cfg.topk_group,
+                             cfg.renormalize, cfg.rsf, self.topk_ids, self.topk_weights, s)
+        capi.moe_append_shared_slots(self.topk_ids, self.topk_weights, E, self.m, self.gate, self.ids2,
+                                     self.w2slots, s)
+        capi.moe_align_sort(self.ids2, self.E2, self.bm, self.sorted_ids, self.block_expert, self.expert_counts,
+                            self.expert_offsets, self.num_padded, s)
+        if probes:
+            probes[0].record(s)
+        capi.moe_stage1_gemm(self.dt, inp["x"], inp.get("x_scale"), self.w13, self.wsc["w13"], self.sorted_ids,
+                             self.block_expert, self.num_padded, T, self.k2, H, I, self.E2, self.bm, self.h,
+                             self.h_scale, self.ws1, s)
+        if probes:
+            probes[1].record(s)
+            probes[2].record(s)
+        capi.moe_stage2_gemm_accumulate(self.dt, self.h, self.h_scale, self.w2, self.wsc["w2"], self.w2slots,
+                                        capi.MOE_DT_F32, self.sorted_ids, self.block_expert, self.num_padded, T,
+                                        self.k2, H, I, self.E2, self.bm, None, None, self.acc_ws, self.out, s)
+        if probes:
+            probes[3].record(s)
+        return self.out
+
+    @property
+    def launches_per_step(self) -> int:
+        """Kernels this library launches per forward()."""
+        prep = 1 if (self.cfg.dtype == "mxfp8" or self.bm >= 32) else 0
+        return (1 if self.gate is not None else 0) + 3 + prep + 2

@@ -122,6 +122,16 @@ def test_quantize_activations_rejects(lib):
 
 
 @no_gpu
+def test_append_shared_slots_rejects(lib):
+    f = lib.moe_append_shared_slots
+    assert f(None, P, 4, 2, 8, 1, None, 0, P, P, None) == -1
+    assert f(P, P, 4, 2, 8, 0, None, 0, P, P, None) == -1          # m >= 1
+    assert f(P, P, 4, 2, 512, 1, None, 0, P, P, None) == -1        # E + m <= 512
+    assert f(P, P, 4, 31, 64, 2, None, 0, P, P, None) == -1        # k + m <= 32
+    assert f(P, P, 4, 2, 8, 1, P, capi.MOE_DT_F32, P, P, None) == -2
+
+
+@no_gpu
 def test_sort_rejects(lib):
     f = lib.moe_align_sort
     assert f(None, 4, 2, 8, 16, P, P, P, P, P, None) == -1
