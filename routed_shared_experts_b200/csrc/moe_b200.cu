@@ -13,6 +13,7 @@
 #include "gate.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 #include "router.cuh"
 #include "sort.cuh"
 
