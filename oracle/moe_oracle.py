@@ -8,8 +8,9 @@ nothing from the product path.
 
 Arithmetic is float64 (numpy), one token / one (token, slot) pair at a time.
 Library primitives used as steps: ``numpy`` matrix-vector products, a stable
-``argsort`` and ``exp``. Number formats (bf16, fp16, fp8 e4m3, ue8m0 block
-scales) are implemented here from their definitions, not taken from a library.
+``argsort`` and ``exp``. Number formats (bf16, fp16, fp8 e4m3, fp4 e2m1, ue8m0
+block scales) are implemented here from their definitions, not taken from a
+library.
 
 Sources (web pages; section names as printed on them):
 
@@ -121,6 +122,37 @@ E4M3_TABLE = np.array([_e4m3_value(c) for c in range(256)], np.float64)
 def e4m3_decode(codes) -> np.ndarray:
     """Decode e4m3 bytes through the 256-entry table of ``_e4m3_value``."""
     return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def _e2m1_value(c: int) -> float:
+    """Value of one OCP E2M1 (FP4) code, bits 0-3 of ``c``: sign bit 3, two
+    exponent bits (bias 1), one mantissa bit; exponent field 0 is subnormal
+    (m/2 * 2**0). Every pattern is a finite number (largest 6, no NaN)."""
+    sign = -1.0 if c & 0x8 else 1.0
+    ef = (c >> 1) & 0x3
+    mf = c & 0x1
+    if ef == 0:
+        return sign * (mf / 2.0)
+    return sign * (1.0 + mf / 2.0) * 2.0 ** (ef - 1)
+
+
+E2M1_TABLE = np.array([_e2m1_value(c) for c in range(16)], np.float64)
+
+
+def e2m1_unpack(packed) -> np.ndarray:
+    """Codes [..., 2n] of e2m1 values stored two per byte [..., n]: element 2j
+    in bits 0-3 of byte j, element 2j+1 in bits 4-7 (the storage order of the
+    MXFP4 weights)."""
+    b = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """Decode e2m1 codes (one per byte, bits 0-3) through ``_e2m1_value``."""
+    return E2M1_TABLE[np.asarray(codes, dtype=np.uint8) & 0xF]
 
 
 def bf16_bits_decode(bits) -> np.ndarray:
@@ -501,9 +533,16 @@ def expert_forward(x_t, w13, w2, I: int, hmode: str, s_x=1.0, s_w13=1.0, s_w2=1.
 def decode_operand(t, fmt: str, scale=None):
     """Float64 values of a stored operand. fmt: 'bf16' / 'fp16' (uint16 bit
     patterns or torch tensors of that dtype), 'fp8' (uint8 e4m3 codes; a
-    per-tensor or per-row scale is applied by the caller, after the matmul), or
-    'mxfp8' (uint8 codes with ue8m0 bytes per 32 columns in ``scale``)."""
+    per-tensor or per-row scale is applied by the caller, after the matmul),
+    'mxfp8' (uint8 codes with ue8m0 bytes per 32 columns in ``scale``), or
+    'mxfp4' (e2m1 codes two per byte, ``e2m1_unpack``, with ue8m0 bytes per 32
+    unpacked columns in ``scale``)."""
     a = _as_numpy(t)
+    if fmt == "mxfp4":
+        v = e2m1_decode(e2m1_unpack(a))
+        sc = ue8m0_decode(_as_numpy(scale))
+        n = v.shape[-1]
+        return (v.reshape(v.shape[:-1] + (n // 32, 32)) * sc[..., None]).reshape(v.shape)
     if fmt in ("bf16", "fp16"):
         if a.dtype == np.uint16:
             return bf16_bits_decode(a) if fmt == "bf16" else fp16_bits_decode(a)
@@ -563,13 +602,17 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> 
     routed sum and the addend meet before the single bf16 rounding; commit 1: the
     routed scaling factor is already inside w.)
 
-    ``cfg`` keys: T H E top_k I Is dtype ('bf16'|'fp8'|'mxfp8') route
+    ``cfg`` keys: T H E top_k I Is dtype ('bf16'|'fp8'|'mxfp8'|'mxfp4') route
     ('softmax'|'grouped_sigmoid') n_group topk_group rsf renormalize shared_gate.
     ``inp`` keys: logits [T,E] fp32, x, w13 [E,2I,H], w2 [E,H,I], w13s [2Is,H],
     w2s [H,Is], optional correction_bias [E], w_gate [H]; fp8 configs add
     x_scale [T], w13_scale [E], w2_scale [E], w13s_scale [1], w2s_scale [1];
     mxfp8 configs add x_scale [T,H/32], w13_scale [E,2I,H/32], w2_scale
     [E,H,I/32], w13s_scale [2Is,H/32], w2s_scale [H,Is/32] (ue8m0 bytes).
+    mxfp4 configs hold the four weight matrices as e2m1 codes two per byte
+    (K halved in the stored shape) with the same scale arrays; x and the
+    quantisation of h are those of mxfp8 (reading: the pages run MXFP4 weights,
+    vllm PR 65207 commit 3, and fix no activation format).
 
     ``shared_fused``: the shared expert taken as always-selected routed experts
     (vllm-project/vllm PR 61503 "Fused heterogeneous MoE", "Overview"): it is cut
@@ -586,11 +629,12 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> 
     """
     T, H, E, k, I, Is = (cfg[n] for n in ("T", "H", "E", "top_k", "I", "Is"))
     fmt = cfg["dtype"]
+    afmt = "mxfp8" if fmt == "mxfp4" else fmt  # activations and h
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     ids, w = route(cfg, _as_numpy(inp["logits"]), None if inp.get("correction_bias") is None
                    else _as_numpy(inp["correction_bias"]))
 
-    x_all = decode_operand(inp["x"], fmt, inp.get("x_scale") if fmt == "mxfp8" else None)
+    x_all = decode_operand(inp["x"], afmt, inp.get("x_scale") if afmt == "mxfp8" else None)
     if fmt == "fp8":
         s_x = _as_numpy(inp["x_scale"]).astype(np.float64).reshape(-1)
     else:
@@ -606,7 +650,7 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> 
     def weights_of(name, e=None):
         wt = inp[name] if e is None else inp[name][e]
         sc = inp.get(name + "_scale")
-        if fmt == "mxfp8":
+        if fmt in ("mxfp8", "mxfp4"):
             return decode_operand(wt, fmt, sc if e is None else sc[e]), 1.0
         if fmt == "fp8":
             s = _as_numpy(sc).astype(np.float64).reshape(-1)
@@ -629,11 +673,11 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> 
             p2[:, : hi - lo] = w2s[:, lo:hi]
             pieces.append((p13, p2))
         for i, t in enumerate(tokens):
-            addend[i] = sum(g[i] * expert_forward(x_all[t], p13, p2, I, fmt, s_x[t], s13s, s2s)
+            addend[i] = sum(g[i] * expert_forward(x_all[t], p13, p2, I, afmt, s_x[t], s13s, s2s)
                             for p13, p2 in pieces)
     else:
         for i, t in enumerate(tokens):
-            ys = expert_forward(x_all[t], w13s, w2s, Is, fmt, s_x[t], s13s, s2s)
+            ys = expert_forward(x_all[t], w13s, w2s, Is, afmt, s_x[t], s13s, s2s)
             addend[i] = bf16_round(g[i] * ys)
 
     # routed experts: each (token, slot) pair is an independent expert call;
@@ -647,7 +691,7 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False) -> 
         for t in tokens:
             for j in range(k):
                 if ids[t, j] == e:
-                    y = expert_forward(x_all[t], w13e, w2e, I, fmt, s_x[t], s13e, s2e)
+                    y = expert_forward(x_all[t], w13e, w2e, I, afmt, s_x[t], s13e, s2e)
                     contrib[pos[int(t)], j] = w[t, j] * y
     routed = np.zeros((len(tokens), H))
     for j in range(k):

@@ -36,6 +36,81 @@ def test_e4m3_table_matches_torch_float8_for_all_codes():
     assert np.all(both_nan | (ref == ours))
 
 
+def test_e2m1_table_matches_closed_form_landmarks():
+    # OCP MX FP4 E2M1: max normal 0b0111 = 6, min normal 0b0010 = 1, the one
+    # subnormal 0b0001 = 0.5, -0 = 0b1000; no NaN or infinity.
+    t = mo.E2M1_TABLE
+    assert t[0b0111] == 6.0 and t[0b1111] == -6.0
+    assert t[0b0010] == 1.0 and t[0b0001] == 0.5 and t[0b0000] == 0.0
+    assert t[0b1000] == 0.0 and math.copysign(1, t[0b1000]) == -1
+    assert list(t[:8]) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.all(np.isfinite(t))
+
+
+def test_e2m1_table_matches_ml_dtypes_for_all_codes():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    ref = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    ours = mo.e2m1_decode(np.arange(16))
+    assert np.array_equal(ref, ours)
+    assert np.array_equal(np.signbit(ref), np.signbit(ours))
+
+
+def test_e2m1_unpack_puts_element_2j_in_the_low_nibble():
+    assert list(mo.e2m1_unpack(np.array([0x21], np.uint8))) == [1, 2]
+    assert list(mo.e2m1_unpack(np.array([0xF7, 0x08], np.uint8))) == [7, 15, 8, 0]
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, (5, 64)).astype(np.uint8)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    assert np.array_equal(mo.e2m1_unpack(packed), codes)
+
+
+def test_mxfp4_decode_equals_a_scalar_loop():
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(4)
+    rows, K = 3, 96
+    packed = rng.integers(0, 256, (rows, K // 2)).astype(np.uint8)
+    sc = rng.integers(100, 140, (rows, K // 32)).astype(np.uint8)
+    got = mo.decode_operand(packed, "mxfp4", sc)
+    for r in range(rows):
+        for j in range(K):
+            byte = int(packed[r, j // 2])
+            code = (byte >> 4) if j % 2 else (byte & 0xF)
+            v = float(np.array([code], np.uint8).view(ml_dtypes.float4_e2m1fn)[0])
+            assert got[r, j] == v * 2.0 ** (int(sc[r, j // 32]) - 127)
+
+
+def test_mxfp4_layer_equals_the_mxfp8_layer_on_the_same_values():
+    # every e2m1 value is an e4m3 value, so MXFP4 weights re-encoded as e4m3
+    # codes (torch's cast) with the same block scales give the same layer
+    T, H, E, k, I, Is = 6, 64, 4, 2, 32, 32
+    cfg = {"T": T, "H": H, "E": E, "top_k": k, "I": I, "Is": Is, "dtype": "mxfp4", "route": "softmax",
+           "n_group": 1, "topk_group": 1, "rsf": 1.0, "renormalize": True, "shared_gate": False}
+    g = torch.Generator().manual_seed(5)
+
+    def w4(*shape):
+        return torch.randint(0, 256, shape[:-1] + (shape[-1] // 2,), generator=g, dtype=torch.uint8)
+
+    def sc(*shape):
+        return torch.randint(118, 124, shape[:-1] + (shape[-1] // 32,), generator=g, dtype=torch.uint8)
+    x = torch.randn(T, H, generator=g)
+    xq = (x * 8).to(torch.float8_e4m3fn).view(torch.uint8)
+    inp = {"logits": torch.randn(T, E, generator=g), "x": xq, "x_scale": torch.full((T, H // 32), 124, dtype=torch.uint8),
+           "w13": w4(E, 2 * I, H), "w13_scale": sc(E, 2 * I, H), "w2": w4(E, H, I), "w2_scale": sc(E, H, I),
+           "w13s": w4(2 * Is, H), "w13s_scale": sc(2 * Is, H), "w2s": w4(H, Is), "w2s_scale": sc(H, Is),
+           "correction_bias": None}
+    r4 = oracle.moe_layer(cfg, inp)
+    e2m1 = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+    def as_e4m3(packed):
+        lo, hi = packed & 0xF, packed >> 4
+        vals = torch.stack([e2m1[lo.long()], e2m1[hi.long()]], dim=-1).reshape(packed.shape[:-1] + (-1,))
+        return vals.to(torch.float8_e4m3fn).view(torch.uint8)
+    inp8 = dict(inp, **{n: as_e4m3(inp[n]) for n in ("w13", "w2", "w13s", "w2s")})
+    r8 = oracle.moe_layer(dict(cfg, dtype="mxfp8"), inp8)
+    assert np.array_equal(r4["out"], r8["out"]) and np.array_equal(r4["addend"], r8["addend"])
+    assert np.any(r4["out"] != 0)
+
+
 def test_e4m3_rounding_matches_torch_cast_inside_range():
     rng = np.random.default_rng(7)
     v = np.concatenate([rng.normal(0, 1, 20000) * 10.0 ** rng.uniform(-4, 2.6, 20000),
