@@ -184,14 +184,13 @@ def barrier(world: int):
 def algorithmic_bytes(cfg, counts, router_gemm=False, quantize_x=False):
     """Bytes the layer and each GEMM must move at minimum (weights of the
     experts the routing activates, activations in and out once)."""
-    el = 2 if cfg.dtype == "bf16" else 1
     active = int((counts > 0).sum())
     rows = int(counts.sum())
-    w13 = 2 * cfg.I * cfg.H * el
-    w2 = cfg.H * cfg.I * el
-    x = cfg.T * cfg.H * el
+    w13 = synth.matrix_bytes(cfg.dtype, 2 * cfg.I * cfg.H)  # codes + scales
+    w2 = synth.matrix_bytes(cfg.dtype, cfg.H * cfg.I)
+    x = synth.activation_bytes(cfg.dtype, cfg.T, cfg.H)
     out = cfg.T * cfg.H * 2
-    h = rows * cfg.I * 2
+    h = synth.activation_bytes(cfg.dtype, rows, cfg.I)
     s1 = active * w13 + x + h
     s2 = active * w2 + h + out + out + rows * 4  # h in, out, addend in, top-k weights
     shared = synth.shared_weight_bytes(cfg)
@@ -315,6 +314,8 @@ def run_ours(args):
     # and the logits unless the step starts from the router linear, which
     # reads bf16 x (the same tensor for a bf16 layer or with --quantize-x)
     names = ["x_r" if args.quantize_x else "x"]
+    if not args.quantize_x and inp.get("x_scale") is not None:
+        names.append("x_scale")
     if args.router_gemm:
         if cfg.dtype != "bf16" and not args.quantize_x:
             names.append("x_r")
@@ -429,19 +430,34 @@ def run_reference(args):
     c = cfg.as_dict()
     # one unit = one expert MLP of one (token, slot) pair, or one token's shared
     # expert; a token is top_k + 1 units. Steps cycle through the workload.
-    ids, w = oracle.route(c, inp["logits"].numpy(), None)
-    x = oracle.decode_operand(inp["x"], cfg.dtype)
+    cb = inp.get("correction_bias")
+    ids, w = oracle.route(c, inp["logits"].numpy(), None if cb is None else cb.numpy())
+    mx = cfg.dtype in ("mxfp8", "mxfp4")
+    afmt = "mxfp8" if mx else cfg.dtype  # activations and h (MXFP4 layers: MXFP8)
+    x = oracle.decode_operand(inp["x"], afmt, inp["x_scale"] if mx else None)
+    s_x = inp["x_scale"].reshape(-1).double().numpy() if cfg.dtype == "fp8" else None
     units = [(t, j) for t in range(cfg.T) for j in range(-1, cfg.top_k)]
+
+    def wts(name, e=None):
+        """Decoded weights and the fp8 per-matrix scale (1 otherwise)."""
+        t, sc = inp[name], inp.get(name + "_scale")
+        if e is not None:
+            t = t[e]
+        if mx:
+            return oracle.decode_operand(t, cfg.dtype, sc if e is None else sc[e]), 1.0
+        if cfg.dtype == "fp8":
+            return oracle.decode_operand(t, "fp8"), float(sc.reshape(-1)[0 if e is None else e])
+        return oracle.decode_operand(t, cfg.dtype), 1.0
 
     def step(i):
         t, j = units[i % len(units)]
+        sx = 1.0 if s_x is None else float(s_x[t])
         if j < 0:
-            oracle.expert_forward(x[t], oracle.decode_operand(inp["w13s"], cfg.dtype),
-                                  oracle.decode_operand(inp["w2s"], cfg.dtype), cfg.Is, cfg.dtype)
+            (w13, s13), (w2, s2), inter = wts("w13s"), wts("w2s"), cfg.Is
         else:
             e = ids[t, j]
-            oracle.expert_forward(x[t], oracle.decode_operand(inp["w13"][e], cfg.dtype),
-                                  oracle.decode_operand(inp["w2"][e], cfg.dtype), cfg.I, cfg.dtype)
+            (w13, s13), (w2, s2), inter = wts("w13", e), wts("w2", e), cfg.I
+        oracle.expert_forward(x[t], w13, w2, inter, afmt, sx, s13, s2)
 
     for i in range(args.warmup):
         step(i)

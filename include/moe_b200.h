@@ -71,6 +71,14 @@ typedef int moe_status_t;
 #define MOE_DT_FP8_E4M3 2   /* e4m3 codes; fp32 scale per token row of x, per expert of W [6106] */
 #define MOE_DT_MXFP8_E4M3 3 /* e4m3 codes; ue8m0 byte per 32 K elements of every row [6106] */
 #define MOE_DT_F32 4
+/* MXFP4 weights against MXFP8 activations (stage 1 and stage 2 only): W13 and
+ * W2 hold OCP e2m1 codes, two per byte (element 2j in bits 0-3 of byte j,
+ * element 2j+1 in bits 4-7), one ue8m0 byte per 32 K elements of every row,
+ * packed by moe_mx_pack_weight_scales as for MXFP8; x, h and their scales are
+ * exactly the MXFP8 operands. The pages run MXFP4 checkpoints on this layer
+ * ([65207] commit 3: Quark OCP MX MoE method); they fix no activation format,
+ * and MXFP8 keeps the stage-2 operand h at 8 bits. */
+#define MOE_DT_MXFP4_E2M1 5
 
 /* Routing modes of moe_router_topk. */
 #define MOE_ROUTE_SOFTMAX 0
@@ -116,8 +124,8 @@ size_t moe_stage2_workspace_bytes(int T, int H);
  *    (x's element type), which the GEMM then reads with one TMA box per
  *    stage instead of gathering rows four at a time (identity routing reads x
  *    itself and leaves this part unused);
- *  - MOE_DT_MXFP8_E4M3: the token scale bytes placed in 512-byte tiles, one
- *    per (token block, 128 columns of H).
+ *  - MOE_DT_MXFP8_E4M3 / MOE_DT_MXFP4_E2M1: the token scale bytes placed in
+ *    512-byte tiles, one per (token block, 128 columns of H).
  * The caller zeroes it ONCE after allocating it; each complete call leaves the
  * counters at zero. */
 size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int I, int block_m);
@@ -260,12 +268,14 @@ moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, vo
  * rows gathered by TMA (block_m 16), or copied into sorted order by a
  * preparation kernel launched first on `stream` (block_m >= 32; MXFP8 token
  * scales always), then read one box per stage.
- *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3 or MOE_DT_MXFP8_E4M3.
+ *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3 or
+ *              MOE_DT_MXFP4_E2M1 (which reads as MXFP8 below except for W13).
  *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8), ue8m0 bytes
  *              [T,H/32] row-major (MXFP8), or NULL (BF16).
  *   w13        [E,2I,H]: rows 0..I-1 gate, I..2I-1 up (K = H contiguous);
  *              w13_scale fp32 [E] (FP8), the packed scale tiles of
- *              moe_mx_pack_weight_scales(0, ...) (MXFP8), or NULL.
+ *              moe_mx_pack_weight_scales(0, ...) (MXFP8, MXFP4), or NULL.
+ *              MXFP4: e2m1 codes, H/2 bytes per row, 32-byte aligned.
  *   sorted_ids / block_expert / num_padded: from moe_align_sort with the same
  *              block_m. sorted_ids == NULL selects identity routing (row r =
  *              token r, expert 0, rows padded to a multiple of block_m; used
@@ -304,8 +314,9 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
  * addend, rounds once to bf16, writes out and re-zeroes its workspace slice.
  *   dtype       as stage 1; h / h_scale are stage 1's outputs.
  *   w2          [E,H,I] (K = I contiguous); w2_scale fp32 [E] (FP8), the
- *               tiles of moe_mx_pack_weight_scales(1, ...) (MXFP8; the block
- *               scales enter the tensor-core MMA), or NULL.
+ *               tiles of moe_mx_pack_weight_scales(1, ...) (MXFP8, MXFP4; the
+ *               block scales enter the tensor-core MMA), or NULL. MXFP4: e2m1
+ *               codes, I/2 bytes per row, 32-byte aligned.
  *   weights     [T*k] per slot f (routing weights, scale folded in), dtype
  *               weights_dtype = MOE_DT_F32, or MOE_DT_BF16 / MOE_DT_FP16 (the
  *               shared gate's output); NULL = 1.0.

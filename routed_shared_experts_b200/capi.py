@@ -14,9 +14,12 @@ import os
 import torch
 
 MOE_OK = 0
-MOE_DT_BF16, MOE_DT_FP16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3, MOE_DT_F32 = 0, 1, 2, 3, 4
+MOE_DT_BF16, MOE_DT_FP16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3, MOE_DT_F32, MOE_DT_MXFP4_E2M1 = 0, 1, 2, 3, 4, 5
 MOE_ROUTE_SOFTMAX, MOE_ROUTE_GROUPED_SIGMOID = 0, 1
+# block-scaled layer formats (MXFP4 layers keep MXFP8 activations)
+MX_FORMATS = ("mxfp8", "mxfp4")
 DTYPES = {"bf16": MOE_DT_BF16, "fp16": MOE_DT_FP16, "fp8": MOE_DT_FP8_E4M3, "mxfp8": MOE_DT_MXFP8_E4M3,
+          "mxfp4": MOE_DT_MXFP4_E2M1,
           "f32": MOE_DT_F32}
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 

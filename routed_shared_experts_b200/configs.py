@@ -8,6 +8,8 @@ Names say what the workload is:
 * ``fp8_a8w8``       T=1024 H=4096 E=64  k=6 I=1408 Is=2816 grouped sigmoid 8/4, rsf 2.5
 * ``mxfp8_prefill``  T=4096 H=7168 E=256 k=8 I=2048 Is=2048 grouped sigmoid 8/4, Zipf logit bias
 * ``fp8_decode_T{n}`` the fp8_a8w8 shapes at T in {1,2,4,...,128}
+* ``mxfp4_decode``   the decode_bf16 shapes (no shared gate) with MXFP4 weights, MXFP8 activations
+* ``mxfp4_prefill``  the mxfp8_prefill shapes with MXFP4 weights, MXFP8 activations
 """
 from __future__ import annotations
 
@@ -24,6 +26,7 @@ class MoEConfig:
     I: int
     Is: int
     dtype: str            # 'bf16' | 'fp8' (per-token x scale, per-expert W scale) | 'mxfp8'
+                          # | 'mxfp4' (e2m1 weights, MXFP8 activations)
     route: str            # 'softmax' | 'grouped_sigmoid'
     seed: int
     block_m: int          # sort padding / token tile of the grouped GEMMs
@@ -56,6 +59,10 @@ MXFP8_PREFILL = MoEConfig("mxfp8_prefill", T=4096, H=7168, E=256, top_k=8, I=204
                           dtype="mxfp8", route="grouped_sigmoid", seed=3, block_m=128,
                           n_group=8, topk_group=4, logit_bias="zipf1.2")
 
+MXFP4_DECODE = MoEConfig("mxfp4_decode", T=32, H=2048, E=128, top_k=8, I=768, Is=512, dtype="mxfp4",
+                         route="softmax", seed=6, block_m=16, logit_bias="normal0.5")
+MXFP4_PREFILL = replace(MXFP8_PREFILL, name="mxfp4_prefill", dtype="mxfp4", seed=5)
+
 SWEEP_T = (1, 2, 4, 8, 16, 32, 64, 128)
 
 
@@ -68,7 +75,7 @@ GATE_K = (1024, 2048, 4096)
 GATE_DTYPES = ("bf16", "fp16")
 GATE_SEED = 4
 
-CONFIGS = {c.name: c for c in (TINY_BF16, DECODE_BF16, FP8_A8W8, MXFP8_PREFILL)}
+CONFIGS = {c.name: c for c in (TINY_BF16, DECODE_BF16, FP8_A8W8, MXFP8_PREFILL, MXFP4_DECODE, MXFP4_PREFILL)}
 CONFIGS.update({fp8_decode(t).name: fp8_decode(t) for t in SWEEP_T})
 
 

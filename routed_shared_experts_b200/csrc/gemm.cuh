@@ -48,7 +48,13 @@ constexpr int kFinBatch = 8;      // stage-2 finalisation: token columns per bat
 // gathers, not HBM, bound the mainloop.
 constexpr int kPermuteMinBN = 32;
 
-enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2 };
+// kMx4: MXFP4 weights (e2m1, two per byte in memory; the tensor map unpacks
+// each 16-element group into 16 bytes of shared memory, so a weight tile has
+// the MXFP8 tile's shape there) against MXFP8 tokens, in the same block-scaled
+// MMA with A declared e2m1.
+enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2, kMx4 = 3 };
+
+__host__ __device__ constexpr bool is_mx(int kind) { return kind == kMx8 || kind == kMx4; }
 
 // Epilogue warpgroups per CTA: two groups take alternate tiles (each with two
 // TMEM accumulators) so a tile's epilogue - atomics to L2 included - overlaps
@@ -56,7 +62,7 @@ enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2 };
 // and MXFP8 keeps two accumulators to leave TMEM room for the scale ring.
 template <int BN, int KIND>
 struct EpiCfg {
-  static constexpr int kGroups = (BN <= 128 && KIND != kMx8) ? 2 : 1;
+  static constexpr int kGroups = (BN <= 128 && !is_mx(KIND)) ? 2 : 1;
   static constexpr int kAcc = 2 * kGroups;
   static constexpr int kThreads = 64 + kEpiThreads * kGroups;
 };
@@ -100,7 +106,7 @@ struct GemmArgs {
 
 template <int BN, int STAGES, int KIND>
 struct GemmSmem {
-  static constexpr bool kMx = KIND == kMx8;
+  static constexpr bool kMx = is_mx(KIND);
   static constexpr int kGroups = EpiCfg<BN, KIND>::kGroups;
   static constexpr int kAcc = EpiCfg<BN, KIND>::kAcc;
   static constexpr int kABytes = kTileM * kTileKBytes;
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
                const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
   using L = GemmSmem<BN, STAGES, KIND>;
   constexpr bool FP8 = KIND == kFp8;
-  constexpr bool MX = KIND == kMx8;
+  constexpr bool MX = is_mx(KIND);
   constexpr int G = L::kGroups;
   constexpr int NACC = L::kAcc;
   constexpr int KE = KIND == kBf16 ? 64 : 128;  // K elements per stage
@@ -497,7 +503,9 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
         if (!ok) break;
         if (lane == 0) {
           pending &= ~(1u << stage);
-          uint32_t bytes = L::kABytes + static_cast<uint32_t>(ncols) * kTileKBytes;
+          // transaction bytes count what the copies read from global memory:
+          // half the shared-memory footprint for the packed e2m1 weight tile
+          uint32_t bytes = (KIND == kMx4 ? L::kABytes / 2 : L::kABytes) + static_cast<uint32_t>(ncols) * kTileKBytes;
           if (MX) bytes += 2 * kSfTile;
           mbar_arrive_expect_tx(&full[stage], bytes);
           if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
             if (MX) {
               // K block kk of the stage: byte kk of each scale column
               const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, ncols, kk), tsfa | sel, tsfb | sel, accum);
+              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, ncols, kk, KIND == kMx4 ? kFmtE2M1 : kFmtE4M3), tsfa | sel, tsfb | sel, accum);
             } else if (FP8) {
               umma_f8(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
             } else {

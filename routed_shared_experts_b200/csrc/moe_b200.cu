@@ -33,6 +33,9 @@ moe_status_t fail_cuda(cudaError_t e, const char* what) {
   } while (0)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+// block-scaled layers: MXFP8 throughout, or MXFP4 weights against MXFP8 tokens
+inline bool is_mx_dtype(int dtype) { return dtype == MOE_DT_MXFP8_E4M3 || dtype == MOE_DT_MXFP4_E2M1; }
 inline cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 inline bool valid_block_m(int bm) { return bm == 16 || bm == 32 || bm == 64 || bm == 128 || bm == 256; }
 
@@ -97,7 +100,7 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
 template <int BN, int KIND>
 constexpr int stages_for() {
   // as many stages as fit in 227 KB of shared memory, one CTA per SM
-  if (KIND == moe::kMx8) return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : 6;
+  if (moe::is_mx(KIND)) return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : 6;
   return BN == 16 ? 12 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
 }
 
@@ -139,7 +142,7 @@ moe_status_t launch_gemm(int bm, const CUtensorMap& ta, const CUtensorMap& tb, c
     case 64: return launch_gemm_bn<64, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
     case 128: return launch_gemm_bn<128, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
     case 256:
-      if constexpr (KIND != moe::kMx8) return launch_gemm_bn<256, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
+      if constexpr (!moe::is_mx(KIND)) return launch_gemm_bn<256, S1, KIND>(ta, tb, tb16, g, max_tiles, s);
       break;
   }
   return MOE_ERR_INVALID_ARG;
@@ -150,6 +153,7 @@ moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CU
                               const CUtensorMap& tb16, const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   if (dtype == MOE_DT_FP8_E4M3) return launch_gemm<S1, moe::kFp8>(bm, ta, tb, tb16, g, max_tiles, s);
   if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, tb16, g, max_tiles, s);
+  if (dtype == MOE_DT_MXFP4_E2M1) return launch_gemm<S1, moe::kMx4>(bm, ta, tb, tb16, g, max_tiles, s);
   return launch_gemm<S1, moe::kBf16>(bm, ta, tb, tb16, g, max_tiles, s);
 }
 
@@ -163,7 +167,7 @@ size_t capacity(int T, int k, int E, int bm) {
 //  * fp8: unquantised fp32 h [rows, I], per-tile row amax [I/64][rows], one
 //    arrival counter per token block, the grid barrier's two words;
 //  * block_m >= kPermuteMinBN: token rows in sorted order [rows, H] (x's type);
-//  * MXFP8: token scale tiles [rows / block_m][H / 128][512].
+//  * MXFP8 / MXFP4: token scale tiles [rows / block_m][H / 128][512].
 struct Stage1Ws {
   size_t amax_off = 0, cnt_off = 0, bar_off = 0, xs_off = 0, xsf_off = 0, total = 0;
   Stage1Ws(int dtype, size_t rows, int H, int I, int bm) {
@@ -178,7 +182,7 @@ struct Stage1Ws {
     xs_off = o;
     if (bm >= moe::kPermuteMinBN) o += up(rows * static_cast<size_t>(H) * (dtype == MOE_DT_BF16 ? 2 : 1));
     xsf_off = o;
-    if (dtype == MOE_DT_MXFP8_E4M3) o += up(rows / bm * static_cast<size_t>(H / 128) * moe::kSfTile);
+    if (is_mx_dtype(dtype)) o += up(rows / bm * static_cast<size_t>(H / 128) * moe::kSfTile);
     total = o;
   }
 };
@@ -311,7 +315,7 @@ size_t moe_stage2_workspace_bytes(int T, int H) {
 }
 
 size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int I, int block_m) {
-  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && dtype != MOE_DT_MXFP8_E4M3) return 0;
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && !is_mx_dtype(dtype)) return 0;
   if (T < 1 || top_k < 1 || E < 1 || H < 1 || I < 1 || !valid_block_m(block_m)) return 0;
   return Stage1Ws(dtype, capacity(T, top_k, E, block_m), H, I, block_m).total;
 }
@@ -437,7 +441,8 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
                              int top_k, int H, int I, int E, int block_m, void* h, void* h_scale, void* ws,
                              moe_stream_t stream) {
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
-  const bool mx = dtype == MOE_DT_MXFP8_E4M3;
+  const bool mx = is_mx_dtype(dtype);
+  const bool w4 = dtype == MOE_DT_MXFP4_E2M1;
   if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!x || !w13 || !h) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
@@ -453,7 +458,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   if (H % (dtype == MOE_DT_BF16 ? 64 : 128) != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
   if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;  // whole 4-block h scale tiles
   if (!aligned16(x) || !aligned16(w13) || !aligned16(h) || (ws && !aligned16(ws)) ||
-      (mx && (!aligned16(x_scale) || !aligned16(w13_scale) || !aligned16(h_scale))))
+      (mx && (!aligned16(x_scale) || !aligned16(w13_scale) || !aligned16(h_scale))) || (w4 && !aligned32(w13)))
     return MOE_ERR_ALIGNMENT;
 
   const bool b16 = dtype == MOE_DT_BF16;
@@ -473,12 +478,14 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   uint8_t* xsf = mx ? wsb + L.xsf_off : nullptr;
   CUtensorMap ta, tb, tb16;
   {
+    // MXFP4: dims count e2m1 elements, strides bytes (two elements a byte);
+    // the 16U4_ALIGN16B type spreads each 8 bytes over 16 in shared memory
+    const size_t wrow = w4 ? static_cast<size_t>(H) / 2 : static_cast<size_t>(H) * es;
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(H), 16, 2, static_cast<cuuint64_t>(I / 16),
                                 static_cast<cuuint64_t>(E)};
-    const cuuint64_t st[4] = {static_cast<cuuint64_t>(H) * es, static_cast<cuuint64_t>(I) * H * es,
-                              16ull * H * es, 2ull * I * H * es};
+    const cuuint64_t st[4] = {wrow, static_cast<cuuint64_t>(I) * wrow, 16ull * wrow, 2ull * I * wrow};
     const cuuint32_t box[5] = {static_cast<cuuint32_t>(ke), 16, 2, 4, 1};
-    moe_status_t r = make_map(&ta, tdt, 5, w13, dims, st, box);
+    moe_status_t r = make_map(&ta, w4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : tdt, 5, w13, dims, st, box);
     if (r != MOE_OK) return r;
   }
   {
@@ -567,7 +574,8 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
                                         int block_m, const void* addend, moe_event_t addend_ready, void* acc_ws,
                                         void* out, moe_stream_t stream) {
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
-  const bool mx = dtype == MOE_DT_MXFP8_E4M3;
+  const bool mx = is_mx_dtype(dtype);
+  const bool w4 = dtype == MOE_DT_MXFP4_E2M1;
   if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
@@ -582,7 +590,8 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
   if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;
   if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)) ||
-      (acc_ws && !aligned16(acc_ws)) || (mx && (!aligned16(h_scale) || !aligned16(w2_scale))))
+      (acc_ws && !aligned16(acc_ws)) || (mx && (!aligned16(h_scale) || !aligned16(w2_scale))) ||
+      (w4 && !aligned32(w2)))
     return MOE_ERR_ALIGNMENT;
 
   const bool b16 = dtype == MOE_DT_BF16;
@@ -594,11 +603,12 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUtensorMap ta, tb, tb16;
   {
+    const size_t wrow = w4 ? static_cast<size_t>(I) / 2 : static_cast<size_t>(I) * es;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(E)};
-    const cuuint64_t st[2] = {static_cast<cuuint64_t>(I) * es, static_cast<cuuint64_t>(H) * I * es};
+    const cuuint64_t st[2] = {wrow, static_cast<cuuint64_t>(H) * wrow};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(moe::kTileM), 1};
-    moe_status_t r = make_map(&ta, tdt, 3, w2, dims, st, box);
+    moe_status_t r = make_map(&ta, w4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : tdt, 3, w2, dims, st, box);
     if (r != MOE_OK) return r;
   }
   {
@@ -678,15 +688,14 @@ moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, cons
                                                   void* out, moe_stream_t stream) {
   // The argument checks of moe_stage2_gemm_accumulate, repeated here so that
   // nothing (not even the clearing memset) is enqueued for an invalid call.
-  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && dtype != MOE_DT_MXFP8_E4M3)
-    return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && !is_mx_dtype(dtype)) return MOE_ERR_UNSUPPORTED_DTYPE;
   if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_DT_BF16 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
-  if (dtype == MOE_DT_MXFP8_E4M3 && (block_m > 128 || I % 128 != 0)) return MOE_ERR_INVALID_ARG;
+  if (is_mx_dtype(dtype) && (block_m > 128 || I % 128 != 0)) return MOE_ERR_INVALID_ARG;
   if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
     return MOE_ERR_UNSUPPORTED_DTYPE;
   if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;

@@ -274,11 +274,16 @@ __device__ __forceinline__ uint64_t plain_rows16_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Operand formats of kind::mxf8f6f4 (instruction descriptor field values).
+constexpr uint32_t kFmtE4M3 = 0;
+constexpr uint32_t kFmtE2M1 = 5;
+
 // Instruction descriptor of kind::mxf8f6f4.block_scale: B scale id [4,6),
-// A/B format e4m3 (0) at [7,10)/[10,13), K-major, N >> 3 at [17,23), scale
-// format ue8m0 (1) at bit 23, M >> 4 at [24,29), A scale id [29,31).
-__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t sf_id) {
-  return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+// A format [7,10) (e4m3 0 or e2m1 5), B format e4m3 (0) at [10,13), K-major,
+// N >> 3 at [17,23), scale format ue8m0 (1) at bit 23, M >> 4 at [24,29),
+// A scale id [29,31), K = 32 (bit 31 clear).
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t sf_id, uint32_t a_fmt = kFmtE4M3) {
+  return (sf_id << 4) | (a_fmt << 7) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
          (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
 }
 

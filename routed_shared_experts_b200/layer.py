@@ -46,6 +46,9 @@ class MoELayer:
         T, H, E, k, I, Is = cfg.T, cfg.H, cfg.E, cfg.top_k, cfg.I, cfg.Is
         self.bm = block_m or cfg.block_m
         self.dt = capi.DTYPES[cfg.dtype]
+        mx = cfg.dtype in capi.MX_FORMATS
+        # activation format of moe_quantize_activations (MXFP4 layers: MXFP8)
+        self.qdt = capi.MOE_DT_MXFP8_E4M3 if mx else self.dt
         bm = self.bm
         cap = capi.sorted_capacity(T, k, E, bm)
         cap_s = capi.sorted_capacity(T, 1, 1, bm)  # identity rows of the shared expert
@@ -69,7 +72,6 @@ class MoELayer:
         self.h = torch.empty((cap, I), dtype=hdt, device=dev)
         self.h_s = torch.empty((cap_s, Is), dtype=hdt, device=dev)
         fp8 = cfg.dtype == "fp8"
-        mx = cfg.dtype == "mxfp8"
         self.h_scale = self.h_scale_s = None
         if fp8:
             self.h_scale = torch.empty(cap, dtype=torch.float32, device=dev)
@@ -77,7 +79,7 @@ class MoELayer:
         elif mx:
             self.h_scale = torch.zeros(capi.mx_h_scale_bytes(T, k, E, I, bm), dtype=torch.uint8, device=dev)
             self.h_scale_s = torch.zeros(capi.mx_h_scale_bytes(T, 1, 1, Is, bm), dtype=torch.uint8, device=dev)
-        # MXFP8 weight scales in the kernels' tile layout (one-off preparation)
+        # MX weight scales in the kernels' tile layout (one-off preparation)
         self.wsc = {}
         for name, which, e, inter in (("w13", 0, E, I), ("w2", 1, E, I), ("w13s", 0, 1, Is), ("w2s", 1, 1, Is)):
             if mx:
@@ -167,7 +169,7 @@ class MoELayer:
         if self.quantize_x:
             # on the side stream, whose stage 1 needs the codes first; the main
             # stream routes and sorts meanwhile and waits only before its stage 1
-            capi.moe_quantize_activations(self.dt, self.inp["x_r"], self.xq, self.xq_scale, self.side)
+            capi.moe_quantize_activations(self.qdt, self.inp["x_r"], self.xq, self.xq_scale, self.side)
             self.ev_q.record(self.side)
         self.shared_expert(self.side)
         self.ev_addend.record(self.side)
@@ -180,7 +182,7 @@ class MoELayer:
         """Kernels this library launches per forward()."""
         cfg = self.cfg
         route = 2 + (1 if self.quantize_x else 0)  # (x quantisation,) top-k, sort
-        mx = cfg.dtype == "mxfp8"
+        mx = cfg.dtype in capi.MX_FORMATS
         prep_routed = 1 if (mx or self.bm >= 32) else 0  # sorted token copy / token scale tiles
         prep_shared = 1 if mx else 0
         gate = 1 if self.gate is not None else 0
@@ -215,17 +217,19 @@ class FusedSharedMoELayer:
         self.bm = bm = block_m or cfg.block_m
         self.dt = capi.DTYPES[cfg.dtype]
         fp8 = cfg.dtype == "fp8"
-        mx = cfg.dtype == "mxfp8"
+        mx = cfg.dtype in capi.MX_FORMATS
+        kd = 2 if cfg.dtype == "mxfp4" else 1  # stored K elements per byte (e2m1: two)
 
         # combined weights [E + m, ...]: routed experts, then the shared pieces
+        # (code 0 is zero in every format)
         w13s, w2s = inp["w13s"], inp["w2s"]
-        p13 = torch.zeros((m, 2 * I, H), dtype=w13s.dtype, device=dev)
-        p2 = torch.zeros((m, H, I), dtype=w2s.dtype, device=dev)
+        p13 = torch.zeros((m, 2 * I, H // kd), dtype=w13s.dtype, device=dev)
+        p2 = torch.zeros((m, H, I // kd), dtype=w2s.dtype, device=dev)
         for v in range(m):
             lo, hi = v * I, min((v + 1) * I, Is)
             p13[v, : hi - lo] = w13s[lo:hi]
             p13[v, I: I + hi - lo] = w13s[Is + lo: Is + hi]
-            p2[v, :, : hi - lo] = w2s[:, lo:hi]
+            p2[v, :, : (hi - lo) // kd] = w2s[:, lo // kd: hi // kd]
         self.w13 = torch.cat([inp["w13"], p13]).contiguous()
         self.w2 = torch.cat([inp["w2"], p2]).contiguous()
         self.wsc = {"w13": None, "w2": None}
@@ -305,5 +309,5 @@ class FusedSharedMoELayer:
     @property
     def launches_per_step(self) -> int:
         """Kernels this library launches per forward()."""
-        prep = 1 if (self.cfg.dtype == "mxfp8" or self.bm >= 32) else 0
+        prep = 1 if (self.cfg.dtype in capi.MX_FORMATS or self.bm >= 32) else 0
         return (1 if self.gate is not None else 0) + 3 + prep + 2

@@ -15,6 +15,11 @@ Input formats (the layer's inputs arrive already in their storage format):
   ``float8_e4m3fn`` cast of the scaled values (clamped to +-448 first).
 * mxfp8 layers: e4m3 codes with one ue8m0 byte per 32 consecutive K elements of
   every row, exponent floor(log2(amax)) - 8 (clamped to [-127, 127]).
+* mxfp4 layers: x as in mxfp8; the weights are drawn directly in storage
+  format, uniform random bytes (two e2m1 codes each, so every one of the 16
+  codes is equally likely) and ue8m0 bytes uniform in {119, 120, 121}
+  (2^-8 .. 2^-6: the codes' rms of 2.9 then gives weights of rms ~0.02).
+  These replace the fp32 normal draws of the weight tensors in the order above.
 
 Router logits are the model's gate linear, which lies before the layer: they are
 made here as fp32 ``x @ W_r`` (from the unrounded draws) plus a per-expert logit
@@ -72,9 +77,17 @@ def _store(v: torch.Tensor, fmt: str, row_dims: int):
         return v.to(torch.bfloat16), None
     if fmt == "fp8":
         return quant_fp8_rows(v, row_dims)
-    if fmt == "mxfp8":
+    if fmt in ("mxfp8", "mxfp4"):  # mxfp4 layers: the MXFP8 activations
         return quant_mx(v)
     raise ValueError(fmt)
+
+
+def draw_mxfp4(rows: int, cols: int, g, device):
+    """Random MXFP4 storage: e2m1 codes [rows, cols/2] (two per byte) and
+    ue8m0 bytes [rows, cols/32]."""
+    codes = torch.randint(0, 256, (rows, cols // 2), generator=g, device=device, dtype=torch.uint8)
+    scales = torch.randint(119, 122, (rows, cols // 32), generator=g, device=device, dtype=torch.uint8)
+    return codes, scales
 
 
 def make_layer_inputs(cfg: MoEConfig, device="cpu") -> dict:
@@ -110,10 +123,15 @@ def make_layer_inputs(cfg: MoEConfig, device="cpu") -> dict:
     if w_gate32 is not None:
         inp["w_gate"] = w_gate32.to(torch.bfloat16)
 
+    def weights(rows, cols):
+        if fmt == "mxfp4":
+            return draw_mxfp4(rows, cols, g, device)
+        return _store(_randn((rows, cols), g, device, std), fmt, 0)
+
     def experts(rows, cols):
         codes, scales = [], []
         for _ in range(E):
-            c, s = _store(_randn((rows, cols), g, device, std), fmt, 0)
+            c, s = weights(rows, cols)
             codes.append(c)
             scales.append(s)
         codes = torch.stack(codes)
@@ -123,8 +141,8 @@ def make_layer_inputs(cfg: MoEConfig, device="cpu") -> dict:
 
     inp["w13"], inp["w13_scale"] = experts(2 * I, H)
     inp["w2"], inp["w2_scale"] = experts(H, I)
-    inp["w13s"], inp["w13s_scale"] = _store(_randn((2 * Is, H), g, device, std), fmt, 0)
-    inp["w2s"], inp["w2s_scale"] = _store(_randn((H, Is), g, device, std), fmt, 0)
+    inp["w13s"], inp["w13s_scale"] = weights(2 * Is, H)
+    inp["w2s"], inp["w2s_scale"] = weights(H, Is)
     inp["correction_bias"] = (_randn((E,), g, device, cfg.correction_bias_std)
                               if cfg.has_correction_bias else None)
     return inp
@@ -144,16 +162,27 @@ def oracle_view(inp: dict) -> dict:
     return {k: (v.detach().cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
 
 
+def matrix_bytes(dtype: str, n: int) -> int:
+    """Stored bytes of one weight matrix of n elements with its scales (fp8:
+    one fp32 scale; MX: one byte per 32 elements)."""
+    codes = {"bf16": 2 * n, "fp8": n, "mxfp8": n, "mxfp4": n // 2}[dtype]
+    return codes + {"bf16": 0, "fp8": 4, "mxfp8": n // 32, "mxfp4": n // 32}[dtype]
+
+
 def weight_bytes_per_expert(cfg: MoEConfig) -> int:
     """Stored bytes of one routed expert (W13 + W2 + their scales)."""
-    el = 2 if cfg.dtype == "bf16" else 1
-    n = 3 * cfg.H * cfg.I
-    sc = {"bf16": 0, "fp8": 8, "mxfp8": n // 32}[cfg.dtype]
-    return n * el + sc
+    return matrix_bytes(cfg.dtype, 2 * cfg.H * cfg.I) + matrix_bytes(cfg.dtype, cfg.H * cfg.I)
 
 
 def shared_weight_bytes(cfg: MoEConfig) -> int:
-    el = 2 if cfg.dtype == "bf16" else 1
-    n = 3 * cfg.H * cfg.Is
-    sc = {"bf16": 0, "fp8": 8, "mxfp8": n // 32}[cfg.dtype]
-    return n * el + sc
+    return matrix_bytes(cfg.dtype, 2 * cfg.H * cfg.Is) + matrix_bytes(cfg.dtype, cfg.H * cfg.Is)
+
+
+def activation_bytes(dtype: str, rows: int, cols: int) -> int:
+    """Stored bytes of a stage operand of rows x cols (x or h) with its scales
+    (fp8: one fp32 per row; MX, MXFP4 layers included: one byte per 32)."""
+    if dtype == "bf16":
+        return 2 * rows * cols
+    if dtype == "fp8":
+        return rows * cols + 4 * rows
+    return rows * cols + rows * cols // 32

@@ -60,6 +60,10 @@ def test_info_calls(lib):
     rows_mx = lib.moe_sorted_capacity(4096, 8, 256, 128)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_MXFP8_E4M3, 4096, 8, 256, 7168, 2048, 128) == \
         up(rows_mx * 7168) + up(rows_mx // 128 * 56 * 512)
+    # MXFP4 weights read the same MXFP8 token operands: same workspace
+    for bm in (16, 32, 128):
+        assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_MXFP4_E2M1, 4096, 8, 256, 7168, 2048, bm) == \
+            lib.moe_stage1_workspace_bytes(capi.MOE_DT_MXFP8_E4M3, 4096, 8, 256, 7168, 2048, bm)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_F32, 32, 8, 128, 2048, 768, 16) == 0
     # MXFP8 scale tiles: 512 bytes per (expert, 128-row tile, 128-column stage)
     assert lib.moe_mx_weight_scale_bytes(0, 256, 7168, 2048) == 256 * (2048 // 64) * (7168 // 128) * 512
@@ -170,6 +174,12 @@ def test_stage1_rejects(lib):
     assert call(H=200) == -4
     assert call(I=100) == -4
     assert call(x=P + 8) == -3
+    w4 = dict(dt=capi.MOE_DT_MXFP4_E2M1, xs=P, ws=P, hs=P, w1=P, H=512, I=128)
+    assert call(dt=capi.MOE_DT_MXFP4_E2M1) == -1                 # scale arrays
+    assert call(**dict(w4, I=192)) == -3                         # whole h scale tiles
+    assert call(**dict(w4, bm=256)) == -1
+    assert call(**dict(w4, H=192)) == -4                         # K stages of 128
+    assert call(**dict(w4, w=P + 16)) == -3                      # e2m1 weights: 32-byte aligned
 
 
 @no_gpu
@@ -188,3 +198,7 @@ def test_stage2_rejects(lib):
     assert call(out=P + 4) == -3
     assert call(add=P + 2) == -3
     assert call(s=None) == -1
+    assert call(dt=capi.MOE_DT_MXFP4_E2M1) == -1                 # h_scale and w2_scale
+    assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, I=192) == -3
+    assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, bm=256) == -1
+    assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, w2=P + 16) == -3
