@@ -120,10 +120,9 @@ size_t moe_stage2_workspace_bytes(int T, int H);
  * `capacity` rows; 256-byte aligned parts, in this order:
  *  - MOE_DT_FP8_E4M3: the unquantised h as fp32 [rows, I], a per-tile row
  *    amax and one arrival counter per token block;
- *  - block_m >= 32: the token rows of x copied into sorted order [rows, H]
- *    (x's element type), which the GEMM then reads with one TMA box per
- *    stage instead of gathering rows four at a time (identity routing reads x
- *    itself and leaves this part unused);
+ *  - the token rows of x copied into sorted order [rows, H] (x's element
+ *    type), which the GEMM then reads with one TMA box per stage (identity
+ *    routing reads x itself and leaves this part unused);
  *  - MOE_DT_MXFP8_E4M3 / MOE_DT_MXFP4_E2M1: the token scale bytes placed in
  *    512-byte tiles, one per (token block, 128 columns of H).
  * The caller zeroes it ONCE after allocating it; each complete call leaves the
@@ -265,9 +264,10 @@ moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, vo
  *     h_r = SiLU(a[0:I]) * a[I:2I]
  * then h_r is stored in the stage-2 operand format ([6106]: quantisation fused
  * after the activation). tcgen05 tensor cores, weights streamed by TMA; token
- * rows gathered by TMA (block_m 16), or copied into sorted order by a
- * preparation kernel launched first on `stream` (block_m >= 32; MXFP8 token
- * scales always), then read one box per stage.
+ * rows (and MXFP8 token scales) copied into sorted order by a preparation
+ * kernel launched first on `stream`, then read one box per stage. The
+ * preparation kernel records device error 3 for a sorted slot id that is
+ * neither a slot nor the padding value T*top_k.
  *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3 or
  *              MOE_DT_MXFP4_E2M1 (which reads as MXFP8 below except for W13).
  *   x          [T,H] bf16 or e4m3 codes; x_scale fp32 [T] (FP8), ue8m0 bytes
@@ -292,8 +292,7 @@ moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, vo
  *              moe_mx_pack_weight_scales with the block_m rows of one token
  *              block per tile. NULL for BF16.
  *   ws         moe_stage1_workspace_bytes(...) bytes, zeroed once by the
- *              caller; may be NULL only when that size is 0 (BF16 with
- *              block_m 16, or BF16 identity routing).
+ *              caller; may be NULL only for BF16 identity routing.
  * Checks: H % 64 == 0 (bf16) / % 128 == 0 (fp8, MXFP8), I % 64 == 0 (% 128
  * for MXFP8), block_m in {16,32,64,128,256} (<= 128 for MXFP8), 16-byte
  * aligned x, w13, h, ws and the MXFP8 scale arrays. */

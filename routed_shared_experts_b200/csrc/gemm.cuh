@@ -5,7 +5,7 @@
 //
 //   warp 0      TMA producer: weight tile (128 rows x 128 K-bytes) and token
 //               tile (BN rows x 128 K-bytes) per pipeline stage. Stage-1 token
-//               rows are gathered from x by TMA gather4 through sorted_ids.
+//               rows come from a copy of x in sorted order (k_stage1_prep).
 //               MXFP8 adds the stage's two 512-byte scale tiles.
 //   warp 1      TMEM allocator + MMA issuer (one thread): tcgen05.mma with the
 //               weights as A (M = 128) and the tokens as B (N = BN), fp32
@@ -42,12 +42,6 @@ constexpr int kEpiThreads = 128;  // one epilogue warpgroup
 constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
 constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)
 constexpr int kFinBatch = 8;      // stage-2 finalisation: token columns per batch of loads
-// Stage 1 with a sorted token tile of at least this many rows reads its token
-// rows from a copy in sorted order (k_stage1_prep) with one 2-D box per stage:
-// tile::gather4 moves 4 rows per instruction, and at 32 rows per stage the
-// gathers, not HBM, bound the mainloop.
-constexpr int kPermuteMinBN = 32;
-
 // kMx4: MXFP4 weights (e2m1, two per byte in memory; the tensor map unpacks
 // each 16-element group into 16 bytes of shared memory, so a weight tile has
 // the MXFP8 tile's shape there) against MXFP8 tokens, in the same block-scaled
@@ -58,11 +52,12 @@ __host__ __device__ constexpr bool is_mx(int kind) { return kind == kMx8 || kind
 
 // Epilogue warpgroups per CTA: two groups take alternate tiles (each with two
 // TMEM accumulators) so a tile's epilogue - atomics to L2 included - overlaps
-// the next tiles' main loop. 256-token tiles fill TMEM with two accumulators,
-// and MXFP8 keeps two accumulators to leave TMEM room for the scale ring.
+// the next tiles' main loop. 256-token tiles fill TMEM with two accumulators;
+// block-scaled tiles keep two from 64 tokens on (TMEM room for the scale ring
+// at 128, registers for the held h values at 64).
 template <int BN, int KIND>
 struct EpiCfg {
-  static constexpr int kGroups = (BN <= 128 && !is_mx(KIND)) ? 2 : 1;
+  static constexpr int kGroups = (is_mx(KIND) ? BN <= 32 : BN <= 128) ? 2 : 1;
   static constexpr int kAcc = 2 * kGroups;
   static constexpr int kThreads = 64 + kEpiThreads * kGroups;
 };
@@ -72,8 +67,6 @@ struct GemmArgs {
   const int32_t* block_expert;
   const int32_t* num_padded;
   int identity_rows;  // identity routing: rows padded to BN
-  int b_tile;         // stage 1: 1 = token rows are one 2-D box at row blk*BN of tmB (identity routing
-                      // over x, or the sorted copy); 0 = gathered from x four rows per tile::gather4
   int cap_blocks;     // token blocks the sorted buffers can hold
   int T, top_k, H, I;
   int n_mt;    // weight tiles per token block
@@ -117,10 +110,10 @@ struct GemmSmem {
   // full[S], empty[S], acc_full[A], acc_empty[A], drain
   static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
-  // tmem slot, abort flag, grid-barrier flag, pad word, producer rows[BN]; then per epilogue
-  // group: ok flag + 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
+  // tmem slot, abort flag, grid-barrier flag, pad word; then per epilogue group: ok flag +
+  // 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
   static constexpr int kGroupWords = 4 + 7 * BN;
-  static constexpr int kMiscBytes = 16 + BN * 4 + kGroups * kGroupWords * 4;
+  static constexpr int kMiscBytes = 16 + kGroups * kGroupWords * 4;
   static constexpr int kBytes = kMiscOffset + kMiscBytes + 1024;  // + alignment slack
   static constexpr int kAccCols = kAcc * BN;
   static constexpr int kSfCol = kAccCols;  // first column of the scale ring
@@ -263,13 +256,16 @@ __host__ __device__ constexpr int sf_tile_offset(int n, int kb) { return (n % 32
 // Stage-1 operand preparation, run before the GEMM on the same stream.
 // Row r of the sorted order (slot f = sorted_ids[r], token f / top_k; with
 // identity routing token r) gets
-//  * xs: a copy of its token's x row (sorted token tiles of kPermuteMinBN
-//    rows or more), so that the GEMM loads BN rows with one box;
+//  * xs: a copy of its token's x row (routed layers), so that the GEMM loads
+//    BN rows with one box per stage (tile::gather4 from x, four rows per
+//    instruction, bounded the main loop at every tile size);
 //  * xsf (MXFP8): its token's ue8m0 scale bytes, placed in the 512-byte tile
 //    of (token block r / bm, stage c) at sf_tile_offset(r % bm, 0..3), the
 //    layout the MMA's scale copy takes, so that the GEMM loads one tile per
 //    stage as it does for the weights.
-// Padding rows are skipped: the MMA column of a padding row is never read.
+// Padding rows are skipped: the MMA column of a padding row is never read. A
+// slot id that is neither a slot nor the padding value T * top_k sets
+// kErrSlotRange.
 struct PrepArgs {
   const uint8_t* x;           // [T][row_bytes]
   const uint8_t* x_scale;     // MXFP8: [T][H / 32]
@@ -294,6 +290,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) k_stage1_prep(const PrepArgs 
     } else {
       const int f = a.sorted_ids[r];
       if (f >= 0 && f < slots) t = f / a.top_k;
+      else if (f != slots && lane == 0) set_device_error(kErrSlotRange);
     }
     if (t < 0) continue;
     if (a.xs) {
@@ -436,8 +433,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
   uint64_t* drain = acc_empty + NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* rows_sm = reinterpret_cast<int*>(tmem_slot + 4);
-  int* group_base = rows_sm + BN;
+  int* group_base = reinterpret_cast<int*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -482,17 +478,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
       const int mt = tile - blk * g.n_mt;
       const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
       const int ncols = block_cols<BN>(g, blk, lane);  // token rows this tile loads and multiplies
-      if (S1 && !g.b_tile) {
-        for (int i = lane; i < BN; i += 32) {
-          const int r = blk * BN + i;
-          int row = 0;
-          const int f = g.sorted_ids[r];
-          if (f >= 0 && f < slots) row = f / g.top_k;
-          else if (f != slots) set_device_error(kErrSlotRange);
-          rows_sm[i] = row;
-        }
-        __syncwarp();
-      }
       for (int kb = 0; kb < g.num_kb; ++kb) {
         uint8_t* a_dst = smem + stage * L::kStageBytes;
         uint8_t* b_dst = a_dst + L::kABytes;
@@ -511,7 +496,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
           else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
           // token rows as one box when the tile is full (B from x, the sorted copy, or h)
-          if ((!S1 || g.b_tile) && ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+          if (ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
           if (MX) {
             const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
             bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
@@ -522,15 +507,9 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
         }
         __syncwarp();
-        // the other token-row loads, issued by the lanes of the warp (the
-        // barrier was armed above with the stage's full byte count)
-        if (S1 && !g.b_tile) {
-          // four rows per gather
-          for (int q = lane; q < ncols / 4; q += 32)
-            tma_gather4(b_dst + q * 4 * kTileKBytes, &tmB, &full[stage], kb * KE, rows_sm[4 * q],
-                        rows_sm[4 * q + 1], rows_sm[4 * q + 2], rows_sm[4 * q + 3], pol_x);
-        } else if (ncols < BN) {
-          // a short tile: 16-row boxes
+        // a short tile: its token rows in 16-row boxes, issued by the lanes of
+        // the warp (the barrier was armed above with the stage's full byte count)
+        if (ncols < BN) {
           for (int q = lane; q < ncols / 16; q += 32)
             tma_load_2d(b_dst + q * 16 * kTileKBytes, &tmB16, &full[stage], kb * KE, blk * BN + q * 16, pol_x);
         }

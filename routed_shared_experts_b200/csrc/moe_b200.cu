@@ -166,7 +166,7 @@ size_t capacity(int T, int k, int E, int bm) {
 // Stage-1 workspace, 256-byte aligned parts:
 //  * fp8: unquantised fp32 h [rows, I], per-tile row amax [I/64][rows], one
 //    arrival counter per token block, the grid barrier's two words;
-//  * block_m >= kPermuteMinBN: token rows in sorted order [rows, H] (x's type);
+//  * routed stage 1: token rows in sorted order [rows, H] (x's type);
 //  * MXFP8 / MXFP4: token scale tiles [rows / block_m][H / 128][512].
 struct Stage1Ws {
   size_t amax_off = 0, cnt_off = 0, bar_off = 0, xs_off = 0, xsf_off = 0, total = 0;
@@ -180,7 +180,7 @@ struct Stage1Ws {
       o = bar_off + 256;
     }
     xs_off = o;
-    if (bm >= moe::kPermuteMinBN) o += up(rows * static_cast<size_t>(H) * (dtype == MOE_DT_BF16 ? 2 : 1));
+    o += up(rows * static_cast<size_t>(H) * (dtype == MOE_DT_BF16 ? 2 : 1));
     xsf_off = o;
     if (is_mx_dtype(dtype)) o += up(rows / bm * static_cast<size_t>(H / 128) * moe::kSfTile);
     total = o;
@@ -449,8 +449,8 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     return MOE_ERR_INVALID_ARG;
   if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
   if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  // routed tiles of kPermuteMinBN rows or more read a sorted copy of the token rows
-  const bool permute = sorted_ids && block_m >= moe::kPermuteMinBN;
+  // routed tiles read a copy of the token rows in sorted order
+  const bool permute = sorted_ids != nullptr;
   if (fp8 && (!x_scale || !w13_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
   if (mx && (!x_scale || !w13_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
   if ((fp8 || mx || permute) && !ws) return MOE_ERR_INVALID_ARG;
@@ -489,31 +489,25 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     if (r != MOE_OK) return r;
   }
   {
-    // token rows: one [block_m x 128 B] box per stage from x (identity
-    // routing; rows past T read as zeros) or from the sorted copy; else
-    // single rows of x for tile::gather4
-    // (tb16: the same rows in 16-row boxes, for tiles with fewer token rows)
-    const bool tile = permute || !sorted_ids;
+    // token rows: one [block_m x 128 B] box per stage from the sorted copy,
+    // or from x itself with identity routing (rows past T read as zeros);
+    // tb16: the same rows in 16-row boxes, for tiles with fewer token rows
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), permute ? static_cast<cuuint64_t>(rows_cap)
                                                                     : static_cast<cuuint64_t>(T)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
     const void* base = permute ? static_cast<const void*>(xs) : x;
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), tile ? static_cast<cuuint32_t>(block_m) : 1u};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
     moe_status_t r = make_map(&tb, tdt, 2, base, dims, st, box);
     if (r != MOE_OK) return r;
-    tb16 = tb;
-    if (tile) {
-      const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
-      r = make_map(&tb16, tdt, 2, base, dims, st, box16);
-      if (r != MOE_OK) return r;
-    }
+    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
+    r = make_map(&tb16, tdt, 2, base, dims, st, box16);
+    if (r != MOE_OK) return r;
   }
   moe::GemmArgs g{};
   g.sorted_ids = sorted_ids;
   g.block_expert = block_expert;
   g.num_padded = num_padded;
   g.identity_rows = cap_blocks * block_m;
-  g.b_tile = (permute || !sorted_ids) ? 1 : 0;
   g.cap_blocks = cap_blocks;
   g.T = T;
   g.top_k = top_k;

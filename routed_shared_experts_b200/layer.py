@@ -183,7 +183,7 @@ class MoELayer:
         cfg = self.cfg
         route = 2 + (1 if self.quantize_x else 0)  # (x quantisation,) top-k, sort
         mx = cfg.dtype in capi.MX_FORMATS
-        prep_routed = 1 if (mx or self.bm >= 32) else 0  # sorted token copy / token scale tiles
+        prep_routed = 1  # sorted token copy (+ MX token scale tiles)
         prep_shared = 1 if mx else 0
         gate = 1 if self.gate is not None else 0
         return route + prep_routed + 2 + gate + prep_shared + 2
@@ -309,5 +309,5 @@ class FusedSharedMoELayer:
     @property
     def launches_per_step(self) -> int:
         """Kernels this library launches per forward()."""
-        prep = 1 if (self.cfg.dtype in capi.MX_FORMATS or self.bm >= 32) else 0
+        prep = 1  # sorted token copy (+ MX token scale tiles)
         return (1 if self.gate is not None else 0) + 3 + prep + 2

@@ -46,17 +46,16 @@ def test_info_calls(lib):
     assert lib.moe_sorted_capacity(5, 3, 7, 64) == 512  # 15 + 441 = 456 -> 512
     assert lib.moe_stage2_workspace_bytes(32, 2048) == 32 * 2048 * 4 + 32 * 16 * 4
     # stage-1 workspace, 256-byte aligned parts: fp8 fp32 h + per-tile amax +
-    # block counters + grid barrier; sorted token rows when block_m >= 32; MXFP8
-    # token scale tiles
+    # block counters + grid barrier; sorted token rows; MXFP8 token scale tiles
     rows = lib.moe_sorted_capacity(1024, 6, 64, 128)
     up = lambda v: (v + 255) // 256 * 256  # noqa: E731
     want = up(rows * 1408 * 4) + up(22 * rows * 4) + up(rows // 128 * 4) + 256 + up(rows * 4096)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 1024, 6, 64, 4096, 1408, 128) == want
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 1024, 6, 64, 4096, 1408, 128) == up(rows * 4096 * 2)
-    assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 32, 8, 128, 2048, 768, 16) == 0
     rows16 = lib.moe_sorted_capacity(32, 8, 128, 16)
+    assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_BF16, 32, 8, 128, 2048, 768, 16) == up(rows16 * 2048 * 2)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_FP8_E4M3, 32, 8, 128, 2048, 768, 16) == \
-        up(rows16 * 768 * 4) + up(12 * rows16 * 4) + up(rows16 // 16 * 4) + 256
+        up(rows16 * 768 * 4) + up(12 * rows16 * 4) + up(rows16 // 16 * 4) + 256 + up(rows16 * 2048)
     rows_mx = lib.moe_sorted_capacity(4096, 8, 256, 128)
     assert lib.moe_stage1_workspace_bytes(capi.MOE_DT_MXFP8_E4M3, 4096, 8, 256, 7168, 2048, 128) == \
         up(rows_mx * 7168) + up(rows_mx // 128 * 56 * 512)
@@ -157,18 +156,19 @@ def test_stage1_rejects(lib):
     f = lib.moe_stage1_gemm
 
     def call(dt=0, x=P, xs=None, w=P, ws=None, s=P, be=P, npd=P, T=4, k=2, H=256, I=128, E=8, bm=16, h=P, hs=None,
-             w1=None):
+             w1=P):
         return f(dt, x, xs, w, ws, s, be, npd, T, k, H, I, E, bm, h, hs, w1, None)
     assert call(dt=capi.MOE_DT_F32) == -2
     assert call(x=None) == -1
     assert call(bm=24) == -1
     assert call(be=None) == -1
     assert call(s=None) == -1                       # identity routing needs top_k == 1
-    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales, h_scale and the workspace
-    assert call(bm=32) == -1                        # sorted token rows need the workspace
+    assert call(dt=capi.MOE_DT_FP8_E4M3) == -1      # fp8 needs scales and h_scale
+    assert call(w1=None) == -1                      # sorted token rows need the workspace
+    assert call(s=None, k=1, w1=None, H=200) == -4  # identity routing needs none
     assert call(dt=capi.MOE_DT_FP8_E4M3, xs=P, ws=P, hs=P, w1=P, H=192) == -4  # fp8 K must be 128-aligned
     assert call(dt=capi.MOE_DT_MXFP8_E4M3) == -1      # MXFP8 needs its scale arrays
-    assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, H=512, I=128) == -1  # token scale tiles: workspace
+    assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, H=512, I=128, w1=None) == -1  # workspace
     assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, w1=P, H=512, I=192) == -3  # whole h scale tiles
     assert call(dt=capi.MOE_DT_MXFP8_E4M3, xs=P, ws=P, hs=P, w1=P, H=512, I=128, bm=256) == -1
     assert call(H=200) == -4
