@@ -75,7 +75,7 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-GEMM_SOURCES = ("gemm.cuh", "ptx.cuh")  # the grouped-GEMM kernel's own sources
+GEMM_SOURCES = ("gemm.cuh", "ptx.cuh", "moe_b200.cu")  # the GEMM kernels and the launcher that picks their instances
 
 
 def src_hash() -> str:

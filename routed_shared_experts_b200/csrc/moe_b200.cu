@@ -99,9 +99,13 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
 
 template <int BN, int KIND>
 constexpr int stages_for() {
-  // as many stages as fit in 227 KB of shared memory, one CTA per SM
+  // as many stages as fit in 227 KB of shared memory, one CTA per SM, except
+  // bf16 / fp8 16-token tiles: six stages (108 KB of operands in flight per SM)
+  // streamed the weights faster than twelve (decode step 152.3 -> 150.4 us
+  // bf16, 194.5 -> 182.6 us fp8 at T = 32), as a bulk-copy stream also peaks at
+  // 64-100 KB in flight per SM and loses DRAM bandwidth beyond
   if (moe::is_mx(KIND)) return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : 6;
-  return BN == 16 ? 12 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
+  return BN == 16 ? 6 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
 }
 
 template <int BN, bool S1, int KIND>
