@@ -50,15 +50,18 @@ enum Kind : int { kBf16 = 0, kFp8 = 1, kMx8 = 2, kMx4 = 3 };
 
 __host__ __device__ constexpr bool is_mx(int kind) { return kind == kMx8 || kind == kMx4; }
 
-// Epilogue warpgroups per CTA: two groups take alternate tiles (each with two
-// TMEM accumulators) so a tile's epilogue - atomics to L2 included - overlaps
-// the next tiles' main loop. 256-token tiles fill TMEM with two accumulators;
-// block-scaled tiles keep two from 64 tokens on (TMEM room for the scale ring
-// at 128, registers for the held h values at 64).
-template <int BN, int KIND>
+// Epilogue warpgroups per CTA: two groups take alternate tiles so a tile's
+// epilogue - atomics to L2 included - overlaps the next tiles' main loop, over
+// a ring of TMEM accumulators (two per group where they fit). 256-token tiles
+// fill TMEM with two accumulators and one group. Block-scaled stage 1 keeps
+// one group from 64 tokens on (registers for the held h values); block-scaled
+// stage 2 at 128 tokens shares three accumulators between its two groups, the
+// scale ring taking TMEM's last columns.
+template <int BN, int KIND, bool S1>
 struct EpiCfg {
-  static constexpr int kGroups = (is_mx(KIND) ? BN <= 32 : BN <= 128) ? 2 : 1;
-  static constexpr int kAcc = 2 * kGroups;
+  static constexpr bool kMxWide = is_mx(KIND) && BN == 128 && !S1;
+  static constexpr int kGroups = (is_mx(KIND) ? (BN <= 32 || !S1) : BN <= 128) ? 2 : 1;
+  static constexpr int kAcc = kMxWide ? 3 : 2 * kGroups;
   static constexpr int kThreads = 64 + kEpiThreads * kGroups;
 };
 
@@ -97,11 +100,11 @@ struct GemmArgs {
   __nv_bfloat16* out;
 };
 
-template <int BN, int STAGES, int KIND>
+template <int BN, int STAGES, int KIND, bool S1>
 struct GemmSmem {
   static constexpr bool kMx = is_mx(KIND);
-  static constexpr int kGroups = EpiCfg<BN, KIND>::kGroups;
-  static constexpr int kAcc = EpiCfg<BN, KIND>::kAcc;
+  static constexpr int kGroups = EpiCfg<BN, KIND, S1>::kGroups;
+  static constexpr int kAcc = EpiCfg<BN, KIND, S1>::kAcc;
   static constexpr int kABytes = kTileM * kTileKBytes;
   static constexpr int kBBytes = BN * kTileKBytes;
   static constexpr int kSfBytes = kMx ? 2 * kSfTile : 0;  // A then B scale tile
@@ -410,10 +413,10 @@ __device__ void quantize_rows_grid(const GemmArgs& g, int rows) {
 }
 
 template <int BN, int STAGES, bool S1, int KIND>
-__global__ void __launch_bounds__(EpiCfg<BN, KIND>::kThreads, 1)
+__global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
-  using L = GemmSmem<BN, STAGES, KIND>;
+  using L = GemmSmem<BN, STAGES, KIND, S1>;
   constexpr bool FP8 = KIND == kFp8;
   constexpr bool MX = is_mx(KIND);
   constexpr int G = L::kGroups;

@@ -112,7 +112,7 @@ template <int BN, bool S1, int KIND>
 moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb16,
                             const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   constexpr int ST = stages_for<BN, KIND>();
-  using L = moe::GemmSmem<BN, ST, KIND>;
+  using L = moe::GemmSmem<BN, ST, KIND, S1>;
   static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
   auto kern = moe::k_moe_gemm<BN, ST, S1, KIND>;
   static std::atomic<int> attr_set[64];
@@ -129,9 +129,9 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
     void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<CUtensorMap*>(&tb16),
                     const_cast<moe::GemmArgs*>(&g)};
     MOE_CK(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
-                                       dim3(moe::EpiCfg<BN, KIND>::kThreads), args, L::kBytes, s));
+                                       dim3(moe::EpiCfg<BN, KIND, S1>::kThreads), args, L::kBytes, s));
   } else {
-    kern<<<grid, moe::EpiCfg<BN, KIND>::kThreads, L::kBytes, s>>>(ta, tb, tb16, g);
+    kern<<<grid, moe::EpiCfg<BN, KIND, S1>::kThreads, L::kBytes, s>>>(ta, tb, tb16, g);
   }
   MOE_CK(cudaGetLastError());
   return MOE_OK;
