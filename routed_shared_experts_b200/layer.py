@@ -18,6 +18,25 @@ from . import capi
 from .configs import MoEConfig
 
 
+def capture_forward(layer, stream=None, steps: int = 1) -> torch.cuda.CUDAGraph:
+    """A CUDA graph of ``steps`` consecutive ``layer.forward(stream)`` calls.
+
+    Replaying it enqueues the same launches on ``stream`` (both streams of the
+    layer included, joined as in ``forward``). The graph reads the layer's input
+    tensors and writes ``layer.out`` in place, so a caller refills the inputs
+    between replays (e.g. copies of the next batch from pinned host memory on
+    the same stream). The layer's workspaces stay valid across replays.
+    """
+    main = stream or torch.cuda.current_stream(layer.device)
+    g = torch.cuda.CUDAGraph()
+    main.wait_stream(torch.cuda.current_stream(layer.device))
+    with torch.cuda.stream(main):
+        with torch.cuda.graph(g, stream=main):
+            for _ in range(steps):
+                layer.forward(main)
+    return g
+
+
 class MoELayer:
     """Device buffers and weights of one layer; ``forward()`` enqueues a step.
 
@@ -176,7 +195,10 @@ class MoELayer:
         self.routed(main, probes=probes, wait_x=self.ev_q if self.quantize_x else None)
         return self.out
 
-    # kernels this library launches per forward()
+    def capture(self, stream=None, steps: int = 1) -> torch.cuda.CUDAGraph:
+        """``capture_forward(self, stream, steps)``: the step as a replayable graph."""
+        return capture_forward(self, stream, steps)
+
     @property
     def launches_per_step(self) -> int:
         """Kernels this library launches per forward()."""
@@ -305,6 +327,10 @@ class FusedSharedMoELayer:
         if probes:
             probes[3].record(s)
         return self.out
+
+    def capture(self, stream=None, steps: int = 1) -> torch.cuda.CUDAGraph:
+        """``capture_forward(self, stream, steps)``: the step as a replayable graph."""
+        return capture_forward(self, stream, steps)
 
     @property
     def launches_per_step(self) -> int:

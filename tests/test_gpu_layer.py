@@ -126,14 +126,11 @@ def test_cuda_graph_replay(cuda_lib):
     layer.forward()
     torch.cuda.synchronize()
     eager = layer.out.float().clone()
-    graph = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
+    graph = layer.capture(s)
     with torch.cuda.stream(s):
-        with torch.cuda.graph(graph, stream=s):
-            layer.forward(s)
-    for _ in range(3):
-        graph.replay()
+        for _ in range(3):
+            graph.replay()
     torch.cuda.synchronize()
     assert capi.device_error() == 0
     assert_close_rms(layer.out.float().cpu().numpy(), eager.cpu().numpy(), BF16_TOL, "graph vs eager",
