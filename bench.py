@@ -40,6 +40,7 @@ METRIC = "MoE layer tokens/s"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "decode_bf16"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 
 def parse():
@@ -73,6 +74,22 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak(dtype: str):
+    """Dense tensor-core peak (TFLOP/s) for the layer's GEMM operand type: the
+    measured sustained bf16 cuBLAS figure (the bench times a long loop), times
+    the nominal 2x of 8-bit over 16-bit operands for fp8 / MX layers."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        bf16, src = float(d.get("bf16_tflops_sustained") or d["bf16_tflops"]), "measured bf16 sustained"
+    else:
+        bf16, src = FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback bf16 sustained"
+    if dtype == "bf16":
+        return bf16, src
+    return 2 * bf16, src + " x 2 (nominal 8-bit / 16-bit ratio)"
 
 
 GEMM_SOURCES = ("gemm.cuh", "ptx.cuh", "moe_b200.cu")  # the GEMM kernels and the launcher that picks their instances
@@ -204,7 +221,10 @@ def algorithmic_bytes(cfg, counts, router_gemm=False, quantize_x=False):
         bf16_x_read = True
     if bf16_x_read:
         layer += cfg.T * cfg.H * 2
-    return {"active_experts": active, "stage1": s1, "stage2": s2, "layer": layer}
+    # GEMM flops of the step (tensor-core work): every routed slot and every
+    # token through the shared expert, gate_up (2I x H) and down (H x I)
+    flops = 6 * rows * cfg.H * cfg.I + 6 * cfg.T * cfg.H * cfg.Is
+    return {"active_experts": active, "stage1": s1, "stage2": s2, "layer": layer, "flops": flops}
 
 
 # ----------------------------------------------------------------- our arm
@@ -301,6 +321,7 @@ def run_ours(args):
         return 1e3 * sum(p[a].elapsed_time(p[b]) for p in probes) / U if K >= U else float("nan")
     s1_us, wait_us, s2_us = avg_us(0, 1), avg_us(1, 2), avg_us(2, 3)
     peak, peak_kind = peaks()
+    tpeak, tpeak_src = tensor_peak(cfg.dtype)
     dom, dom_us = ("stage1", s1_us) if s1_us >= s2_us else ("stage2", s2_us)
     kname = "k_moe_gemm<stage1>" if dom == "stage1" else "k_moe_gemm<stage2>"
     achieved = ab[dom] / (dom_us * 1e-6) / 1e9
@@ -392,7 +413,12 @@ def run_ours(args):
                      "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
                      "bytes_per_launch": ab[dom], "launch_us": dom_us},
         "layer_roofline": {"bytes_per_step": ab["layer"], "t_roof_us": ab["layer"] / (peak * 1e9) * 1e6,
-                           "t_step_us": step_s * 1e6, "frac": ab["layer"] / (peak * 1e9) / step_s},
+                           "t_step_us": step_s * 1e6, "frac": ab["layer"] / (peak * 1e9) / step_s,
+                           "tensor": {"flops_per_step": ab["flops"], "peak_tflops": tpeak, "peak_source": tpeak_src,
+                                      "t_roof_us": ab["flops"] / (tpeak * 1e12) * 1e6,
+                                      "frac": ab["flops"] / (tpeak * 1e12) / step_s},
+                           "binding": "hbm" if ab["layer"] / (peak * 1e9) >= ab["flops"] / (tpeak * 1e12)
+                           else "tensor"},
         "kernels_us": {"stage1": s1_us, "addend_wait": wait_us, "stage2": s2_us,
                        "note": "from the last U steps, whose graph carries timing events"},
         "e2e": {"value": tokens * E2E / (e2e_ms / 1e3), "unit": UNIT,
