@@ -184,12 +184,21 @@ def dist_env():
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of every rank's v (each rank's device time of the same
+    region): the job is as slow as its slowest replica."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps of
+    `tokens_per_rank` tokens, timed as the slowest rank's `ms_max`."""
+    return tokens_per_rank * world * steps / (ms_max / 1e3)
 
 
 def barrier(world: int):
@@ -327,10 +336,9 @@ def run_ours(args):
     achieved = ab[dom] / (dom_us * 1e-6) / 1e9
     traffic = recorded_traffic(kname, cfg.name)
     step_s = ms / 1e3 / K
-    tokens = cfg.T * world
 
-    # e2e through the public API with host buffers: H2D of x and logits from
-    # pinned memory, the five calls, D2H of the output, every step
+    # e2e with host buffers, every step: H2D of the step's inputs from pinned
+    # memory, the step, D2H of its output (StepPipeline below; eager for comparison)
     # step inputs copied from pinned host memory: the activations the step
     # reads (bf16 x when the step quantises it, else x in the layer's format),
     # and the logits unless the step starts from the router linear, which
@@ -392,7 +400,7 @@ def run_ours(args):
 
     result = {
         "metric": METRIC,
-        "value": tokens * K / (ms / 1e3),
+        "value": job_tokens_per_s(cfg.T, world, K, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": K,
@@ -421,12 +429,12 @@ def run_ours(args):
                            else "tensor"},
         "kernels_us": {"stage1": s1_us, "addend_wait": wait_us, "stage2": s2_us,
                        "note": "from the last U steps, whose graph carries timing events"},
-        "e2e": {"value": tokens * E2E / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_tokens_per_s(cfg.T, world, E2E, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": sum(hs.numel() * hs.element_size() for hs in hosts),
                 "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": E2E,
                 "api": "StepPipeline.run: per step H2D copies (pinned) -> graph of the step -> D2H copy (pinned), "
                        "the copies of steps i+1 and i-1 overlapping step i on a copy stream",
-                "eager": {"value": tokens * E2E / (eager_ms / 1e3),
+                "eager": {"value": job_tokens_per_s(cfg.T, world, E2E, eager_ms),
                           "api": "layer.forward() per step (eager C-ABI calls), the same copies serialised with it"}},
         "gpu_launches": K * layer.launches_per_step,
         "clocks": clk,
