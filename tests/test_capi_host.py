@@ -202,3 +202,20 @@ def test_stage2_rejects(lib):
     assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, I=192) == -3
     assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, bm=256) == -1
     assert call(dt=capi.MOE_DT_MXFP4_E2M1, hs=P, w2s=P, w2=P + 16) == -3
+
+
+def test_binding_rejects_host_tensors_before_any_call(lib):
+    """The Python binding only marshals device tensors: a host tensor (whose
+    address a kernel must never see) or a non-tensor is refused in Python."""
+    with pytest.raises(ValueError):
+        capi._ptr(torch.zeros(4))
+    with pytest.raises(TypeError):
+        capi._ptr([0, 1, 2])
+    assert capi._ptr(None) is None
+    ids = torch.zeros((4, 2), dtype=torch.int32)
+    out = torch.zeros(64, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        capi.moe_align_sort(ids, 8, 16, out, out, out, out, out)
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        capi.shared_expert_gate_dot(capi.MOE_DT_BF16, x, x[0], True, torch.zeros(4, dtype=torch.bfloat16))
