@@ -123,6 +123,26 @@ def test_e4m3_rounding_matches_torch_cast_inside_range():
     assert np.array_equal(ours[exact32], ref[exact32])
 
 
+def test_e4m3_rounding_at_every_midpoint_and_its_fp32_neighbours():
+    # For every pair of adjacent non-negative e4m3 values: the midpoint (a tie),
+    # the fp32 numbers just below and just above it, both values, and the fp32
+    # numbers next to them; both signs. A misplaced rounding bit, a wrong tie
+    # rule or a wrong subnormal spacing changes one of these decisions.
+    t = mo.E4M3_TABLE[:0x7F]  # 0 .. 448, increasing
+    mid = ((t[1:] + t[:-1]) / 2).astype(np.float32)
+    pts = [mid, t.astype(np.float32)]
+    for base in (mid, t.astype(np.float32)):
+        pts.append(np.nextafter(base, np.float32(np.inf)))
+        pts.append(np.nextafter(base, np.float32(-np.inf)))
+    v = np.concatenate(pts)
+    v = v[(v >= 0) & (v <= 448)]
+    v = np.concatenate([v, -v]).astype(np.float32)
+    ours = oracle.round_to_format(v.astype(np.float64), oracle.E4M3)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(ours, ref)
+    assert np.array_equal(np.signbit(ours[ours == 0]), np.signbit(ref[ref == 0]))
+
+
 def test_e4m3_ties_to_even_and_saturation():
     # 1.0625 lies midway between 1.0 (mantissa 000) and 1.125 (001): even -> 1.0
     # 1.1875 midway between 1.125 (001) and 1.25 (010): even -> 1.25
