@@ -108,3 +108,11 @@ def test_mx_and_fp8_bytes_count_their_scales():
     assert synth.matrix_bytes("mxfp4", n) == n // 2 + n // 32
     assert synth.activation_bytes("fp8", 10, 4096) == 10 * 4096 + 40
     assert synth.activation_bytes("mxfp4", 10, 4096) == 10 * 4096 + 10 * 128
+
+
+def test_l2_note_is_true_to_the_step_size():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert "come from HBM" in bench.l2_note(0.81e9)
+    assert "may still be in L2" in bench.l2_note(200e6)
+    assert "L2-resident" in bench.l2_note(1.8e6)
