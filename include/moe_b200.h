@@ -116,7 +116,7 @@ size_t moe_sorted_capacity(int T, int top_k, int E, int block_m);
  * zeroes it ONCE after allocating it; each complete call leaves it zeroed. */
 size_t moe_stage2_workspace_bytes(int T, int H);
 
-/* Bytes of the stage-1 workspace for `dtype` (0 when none is needed), for
+/* Bytes of the stage-1 workspace for `dtype` (0 for invalid arguments), for
  * `capacity` rows; 256-byte aligned parts, in this order:
  *  - MOE_DT_FP8_E4M3: the unquantised h as fp32 [rows, I], a per-tile row
  *    amax and one arrival counter per token block;
@@ -129,7 +129,8 @@ size_t moe_stage2_workspace_bytes(int T, int H);
  * counters at zero. */
 size_t moe_stage1_workspace_bytes(int dtype, int T, int top_k, int E, int H, int I, int block_m);
 
-/* Bytes of the packed MXFP8 weight scales of one projection: which = 0 for W13
+/* Bytes of the packed block-scale tiles of one projection's weights (MXFP8 or
+ * MXFP4: one ue8m0 byte per 32 K elements either way): which = 0 for W13
  * ([E,2I,H] weights), which = 1 for W2 ([E,H,I] weights). 0 unless H and I are
  * multiples of 128. */
 size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I);
@@ -138,8 +139,9 @@ size_t moe_mx_weight_scale_bytes(int which, int E, int H, int I);
  * columns); 0 for an unsupported shape. */
 size_t moe_mx_h_scale_bytes(int T, int top_k, int E, int I, int block_m);
 
-/* moe_mx_pack_weight_scales: one-off weight preparation for MXFP8 (no
- * counterpart on the pages; MXFP8 itself is [6106]'s BLOCK_K = 32 format).
+/* moe_mx_pack_weight_scales: one-off weight preparation for MXFP8 and MXFP4
+ * weights (no counterpart on the pages; MXFP8 itself is [6106]'s BLOCK_K = 32
+ * format, and MXFP4 weights carry the same one-byte scale per 32 elements).
  * src holds the ue8m0 scale bytes row-major, [E, rows, K/32] (which = 0: W13,
  * rows = 2I, K = H; which = 1: W2, rows = H, K = I). dst
  * (moe_mx_weight_scale_bytes) receives them as 512-byte tiles, one per
