@@ -44,6 +44,10 @@ def test_info_calls(lib):
     assert lib.moe_status_string(-1) == b"MOE_ERR_INVALID_ARG"
     assert lib.moe_sorted_capacity(32, 8, 128, 16) == 32 * 8 + 128 * 15  # already a multiple of 16
     assert lib.moe_sorted_capacity(5, 3, 7, 64) == 512  # 15 + 441 = 456 -> 512
+    # the library's capacity is the plain bound rounded up to whole blocks
+    import oracle
+    for T, k, E, bm in ((5, 3, 7, 64), (32, 8, 128, 16), (1024, 6, 64, 128), (3, 2, 6, 16)):
+        assert lib.moe_sorted_capacity(T, k, E, bm) == -(-oracle.sorted_capacity(T, k, E, bm) // bm) * bm
     assert lib.moe_stage2_workspace_bytes(32, 2048) == 32 * 2048 * 4 + 32 * 16 * 4
     # stage-1 workspace, 256-byte aligned parts: fp8 fp32 h + per-tile amax +
     # block counters + grid barrier; sorted token rows; MXFP8 token scale tiles

@@ -28,6 +28,25 @@ def test_e4m3_table_matches_closed_form_landmarks():
     assert t[0x07] == 7 * 2.0**-9 and t[0x0F] == 1.875 * 2.0**-6
 
 
+def test_ue8m0_decode_is_a_power_of_two_per_byte():
+    # OCP MX E8M0 scale: byte b stands for 2^(b - 127); 127 is 1.0
+    b = np.arange(255, dtype=np.uint8)
+    v = mo.ue8m0_decode(b)
+    assert v[127] == 1.0 and v[128] == 2.0 and v[126] == 0.5
+    assert v[0] == 2.0**-127 and v[254] == 2.0**127
+    assert np.all(v[1:] / v[:-1] == 2.0)
+
+
+def test_sorted_capacity_bounds_every_padded_sort():
+    # T*k slots plus at most block_m - 1 padding rows for each of E experts;
+    # a sort where every expert holds one slot reaches the bound exactly
+    for T, k, E, bm in ((5, 3, 7, 64), (32, 8, 128, 16), (1, 1, 1, 16), (3, 2, 6, 16)):
+        assert oracle.sorted_capacity(T, k, E, bm) == T * k + E * (bm - 1)
+    ids = np.arange(6, dtype=np.int64).reshape(3, 2)  # 6 experts, one slot each
+    r = oracle.align_sort(ids, 6, 16)
+    assert r["num_padded"] == 6 * 16 == oracle.sorted_capacity(3, 2, 6, 16)
+
+
 def test_e4m3_table_matches_torch_float8_for_all_codes():
     codes = torch.arange(256, dtype=torch.uint8)
     ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
