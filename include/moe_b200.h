@@ -105,6 +105,13 @@ int moe_supports_output_addend(void);
  * 2 = expert id out of range in the sort, 3 = sorted slot id out of range. */
 moe_status_t moe_device_error(int* code, moe_stream_t stream);
 
+/* Self-test of the failure path: launches one CTA whose thread waits, through
+ * the grouped GEMM's own bounded mbarrier wait, on a barrier phase that nothing
+ * completes. After the wait limit (4 s) it records device error 1 and returns;
+ * the context stays usable. Read the code with moe_device_error. Asynchronous
+ * on `stream`. */
+moe_status_t moe_selftest_wait_timeout(moe_stream_t stream);
+
 /* Number of int32 slots the padded sort output may need: T*top_k +
  * E*(block_m - 1) rounded up to a multiple of block_m ("capacity rows").
  * sorted_ids holds this many entries, block_expert this / block_m, and the

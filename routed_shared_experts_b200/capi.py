@@ -31,6 +31,7 @@ SIGNATURES = {
     "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_supports_output_addend": (_I, []),
     "moe_device_error": (_I, [ctypes.POINTER(ctypes.c_int), _P]),
+    "moe_selftest_wait_timeout": (_I, [_P]),
     "moe_sorted_capacity": (_SZ, [_I, _I, _I, _I]),
     "moe_stage2_workspace_bytes": (_SZ, [_I, _I]),
     "moe_stage1_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
@@ -134,6 +135,11 @@ def device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("moe_device_error", lib().moe_device_error(ctypes.byref(code), _stream(stream)))
     return code.value
+
+
+def moe_selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait self-test (device error 1 after ~4 s)."""
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(_stream(stream)))
 
 
 def moe_router_topk(logits, correction_bias, top_k, mode, n_group, topk_group, renormalize,

@@ -15,6 +15,7 @@
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "router.cuh"
+#include "selftest.cuh"
 #include "sort.cuh"
 
 namespace {
@@ -304,6 +305,12 @@ moe_status_t moe_device_error(int* code, moe_stream_t stream) {
   const int zero = 0;
   MOE_CK(cudaMemcpyToSymbol(moe::g_device_error, &zero, sizeof(int)));
   *code = v;
+  return MOE_OK;
+}
+
+moe_status_t moe_selftest_wait_timeout(moe_stream_t stream) {
+  moe::k_selftest_wait_timeout<<<1, 32, 0, as_stream(stream)>>>();
+  MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
 
