@@ -3,6 +3,10 @@ force on tiny inputs, library special cases and invariants. CPU only.
 
 Each test is chosen so that a plausible slip in the oracle (a dropped term, a
 swapped operand, a wrong sign or index, a wrong tie rule) fails it.
+
+Every pin runs twice: against the oracle of record, the plain C++ one
+(oracle/moe_oracle.cpp through oracle/cpp.py), and against the independent
+float64 numpy statement of the same definitions (oracle/moe_oracle.py).
 """
 import itertools
 import math
@@ -11,8 +15,20 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
-from oracle import moe_oracle as mo
+from oracle import cpp as _cpp_oracle
+from oracle import moe_oracle as _np_oracle
+
+oracle = mo = _cpp_oracle  # set per test by the fixture below
+IMPLS = {"cpp": _cpp_oracle, "numpy": _np_oracle}
+
+
+@pytest.fixture(autouse=True, params=sorted(IMPLS))
+def oracle_impl(request):
+    """Runs the test against each oracle implementation (module globals
+    ``oracle`` and ``mo`` name the one under test)."""
+    global oracle, mo
+    oracle = mo = IMPLS[request.param]
+    yield request.param
 
 # ---------------------------------------------------------------- formats
 
@@ -679,3 +695,91 @@ def test_layer_single_expert_is_dense_mlp():
     y = h @ inp["w2"][0].double().T
     np.testing.assert_allclose(r["routed"], y.numpy(), rtol=1e-10, atol=1e-14)
     np.testing.assert_allclose(r["topk_weights"], 1.0)
+
+
+def test_fp8_layer_takes_each_experts_and_each_tokens_own_scale():
+    """fp8 a8w8 (ROCm/aiter PR 6106, "Technical Details": one activation scale
+    per token row, one weight scale per expert) with every expert's W13 and W2
+    scale different (2^(e mod 7) * 1e-3 and 2^((e + 3) mod 5) * 2e-3) and every
+    token's x scale different, against a scalar-loop brute force. Fails if the
+    oracle took s[0] for every expert, swapped the W13 and W2 scales, or
+    indexed the activation scale by slot or sorted row instead of by token."""
+    T, H, E, k, I, Is = 7, 32, 6, 3, 32, 32
+    cfg = dict(_tiny_cfg(T=T, H=H, E=E, top_k=k, I=I, Is=Is), dtype="fp8", shared_gate=False)
+    g = np.random.default_rng(12)
+    codes = lambda *sh: (g.integers(0, 0x70, sh).astype(np.uint8)  # noqa: E731
+                         | (g.integers(0, 2, sh) * 0x80).astype(np.uint8))
+    s13 = np.array([2.0 ** (e % 7) * 1e-3 for e in range(E)])
+    s2 = np.array([2.0 ** ((e + 3) % 5) * 2e-3 for e in range(E)])
+    sx = np.array([0.004 * (1 + 0.37 * t) for t in range(T)])
+    inp = {"logits": g.normal(size=(T, E)).astype(np.float32), "x": codes(T, H), "x_scale": sx,
+           "w13": codes(E, 2 * I, H), "w2": codes(E, H, I), "w13_scale": s13, "w2_scale": s2,
+           "w13s": codes(2 * Is, H), "w2s": codes(H, Is), "w13s_scale": np.array([3e-3]),
+           "w2s_scale": np.array([7e-4]), "correction_bias": None}
+    r = oracle.moe_layer(cfg, inp)
+    x = _np_table_e4m3()[inp["x"]]
+    w13, w2 = _np_table_e4m3()[inp["w13"]], _np_table_e4m3()[inp["w2"]]
+    w13s, w2s = _np_table_e4m3()[inp["w13s"]], _np_table_e4m3()[inp["w2s"]]
+
+    def mlp(xt, a13, a2, inter, sxt, sa, sb):
+        a = [sum(a13[i, c] * xt[c] for c in range(H)) * sxt * sa for i in range(2 * inter)]
+        h = [a[i] / (1 + math.exp(-a[i])) * a[inter + i] for i in range(inter)]
+        amax = max(abs(v) for v in h)
+        s = float(np.float32(amax / 448)) if amax > 0 else 1.0
+        hq = [_e4m3_rn(v / s) * s for v in h]
+        return np.array([sum(a2[o, i] * hq[i] for i in range(inter)) * sb for o in range(H)])
+    lg = inp["logits"]
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-lg[t, e], e))[:k]
+        p = [math.exp(float(lg[t, e]) - float(lg[t, order[0]])) for e in order]
+        wts = [v / sum(p) for v in p]
+        assert list(r["topk_ids"][t]) == order
+        addend = _bf16_rn(mlp(x[t], w13s, w2s, Is, sx[t], 3e-3, 7e-4))
+        routed = sum(wts[j] * mlp(x[t], w13[order[j]], w2[order[j]], I, sx[t], s13[order[j]], s2[order[j]])
+                     for j in range(k))
+        np.testing.assert_allclose(r["addend"][t], addend, rtol=0, atol=0)
+        np.testing.assert_allclose(r["routed"][t], routed, rtol=1e-12, atol=1e-15 * np.max(np.abs(routed)))
+    # the same layer with one scale changed moves exactly the tokens routed to that expert
+    e0 = int(r["topk_ids"][0, 0])
+    bumped = dict(inp, w2_scale=np.where(np.arange(E) == e0, 2 * s2, s2))
+    rb = oracle.moe_layer(cfg, bumped)
+    uses = np.any(r["topk_ids"] == e0, axis=1)
+    moved = np.any(rb["routed"] != r["routed"], axis=1)
+    assert np.array_equal(moved, uses)
+
+
+def _np_table_e4m3():
+    """E4M3 values from the closed form of the format (independent of both
+    oracles): sign * 2^(e-7) * (1 + m/8), subnormal 2^-6 * m/8, NaN at S.1111.111."""
+    t = np.empty(256)
+    for c in range(256):
+        sgn = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 15, c & 7
+        t[c] = math.nan if (e == 15 and m == 7) else sgn * (2.0 ** -6 * m / 8 if e == 0 else 2.0 ** (e - 7) * (1 + m / 8))
+    return t
+
+
+def _e4m3_rn(v):
+    """Nearest E4M3 value (ties to the even code), saturating at 448: scan of
+    the finite non-negative values."""
+    vals = _np_table_e4m3()[:0x7F]
+    a = min(abs(v), 448.0)
+    i = int(np.argmin(np.abs(vals - a)))
+    d = abs(vals[i] - a)
+    cands = [j for j in range(len(vals)) if abs(vals[j] - a) == d]
+    j = [c for c in cands if c % 2 == 0][0] if len(cands) > 1 else cands[0]
+    return math.copysign(vals[j], v)
+
+
+def _bf16_rn(v):
+    """bf16 rounding written from the format (8 significant bits, ties to
+    even by Python's round) for normal-range float64 values."""
+    out = []
+    for x in np.ravel(np.asarray(v, np.float64)):
+        if x == 0:
+            out.append(x)
+            continue
+        _, e = math.frexp(x)  # |x| in [2^(e-1), 2^e): spacing 2^(e-1-7)
+        q = 2.0 ** (e - 8)
+        out.append(round(x / q) * q)
+    return np.array(out).reshape(np.shape(v))
