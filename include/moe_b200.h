@@ -40,6 +40,19 @@
  *     records a code in a device error word read by moe_device_error().
  *   - Layouts are row-major and dense unless stated. T tokens, H hidden, E
  *     routed experts, k = top_k, I expert intermediate size.
+ *   - The grouped GEMMs of 128-token blocks run on CTA pairs (2-CTA
+ *     clusters sharing one M = 256 tensor-core MMA, each SM loading its 128
+ *     weight rows and half of the token rows) when the weight rows split into
+ *     an even number of 128-row tiles (stage 1: I % 128 == 0, except the fp8
+ *     stage 1, whose per-row quantisation follows a grid barrier; stage 2:
+ *     H % 256 == 0); otherwise, and with MOE_B200_PAIR=0 in the environment,
+ *     one CTA per tile. Results do not depend on the choice.
+ *   - Shapes the grouped GEMMs cover (anything else returns MOE_ERR_SHAPE or
+ *     MOE_ERR_ALIGNMENT and launches nothing): H % 128 == 0 (stage 1 with bf16
+ *     operands: H % 64 == 0), I % 64 == 0, and I % 128 == 0 for MXFP8 and
+ *     MXFP4; token blocks (block_m) of 16, 32, 64, 128 or 256 rows (at most
+ *     128 for MXFP8 / MXFP4). Smaller alignments (H % 16, block_m = 8) are
+ *     not supported.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -102,7 +115,9 @@ int moe_supports_output_addend(void);
 
 /* Reads the current device's error word into *code (0 = none) and clears it.
  * Synchronises `stream` first. Codes: 1 = bounded mbarrier wait gave up,
- * 2 = expert id out of range in the sort, 3 = sorted slot id out of range. */
+ * 2 = expert id out of range in the sort, 3 = sorted slot id out of range,
+ * 4 = a block_expert entry outside [0, E) met by a grouped GEMM (the block is
+ * then computed with expert 0's weights, so no access leaves the weights). */
 moe_status_t moe_device_error(int* code, moe_stream_t stream);
 
 /* Self-test of the failure path: launches one CTA whose thread waits, through
@@ -370,7 +385,11 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
  *     moe_last_cuda_error()) and launch nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is kept for the life of the
+ *     process: after a cudaDeviceReset it is stale, so do not call this entry
+ *     point again in a process that has reset the device.
+ *   - `stream` must belong to the current device (MOE_ERR_DEVICE otherwise:
+ *     the array used is the current device's).
  *   - The array is shared by every call on a device and keeps the last call's
  *     contents; each call clears the part it uses on `stream` before its
  *     kernel. Calls whose work overlaps on the GPU (concurrent streams) race

@@ -72,6 +72,7 @@ struct GemmArgs {
   int identity_rows;  // identity routing: rows padded to BN
   int cap_blocks;     // token blocks the sorted buffers can hold
   int T, top_k, H, I;
+  int E;       // experts the weight tensors hold (block_expert entries are checked against it)
   int n_mt;    // weight tiles per token block
   int num_kb;  // K stages per tile
   // stage 1 outputs
@@ -100,13 +101,15 @@ struct GemmArgs {
   __nv_bfloat16* out;
 };
 
-template <int BN, int STAGES, int KIND, bool S1>
+// PAIR: the tile is computed by a CTA pair (one MMA of M = 256); each CTA
+// holds its 128 weight rows and half of the BN token rows of a stage.
+template <int BN, int STAGES, int KIND, bool S1, bool PAIR = false>
 struct GemmSmem {
   static constexpr bool kMx = is_mx(KIND);
   static constexpr int kGroups = EpiCfg<BN, KIND, S1>::kGroups;
   static constexpr int kAcc = EpiCfg<BN, KIND, S1>::kAcc;
   static constexpr int kABytes = kTileM * kTileKBytes;
-  static constexpr int kBBytes = BN * kTileKBytes;
+  static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kTileKBytes;
   static constexpr int kSfBytes = kMx ? 2 * kSfTile : 0;  // A then B scale tile
   static constexpr int kStageBytes = kABytes + kBBytes + kSfBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
@@ -131,6 +134,19 @@ __device__ __forceinline__ float load_weight(const void* w, int dt, int f) {
   if (dt == 4) return static_cast<const float*>(w)[f];
   if (dt == 0) return __bfloat162float(static_cast<const __nv_bfloat16*>(w)[f]);
   return __half2float(static_cast<const __half*>(w)[f]);
+}
+
+// Expert of token block `blk` (0 with identity routing). An entry outside
+// [0, E) - a stale or foreign block_expert buffer - records kErrBlockExpert
+// and reads as expert 0, so that no load or scale lookup leaves the weights.
+__device__ __forceinline__ int block_expert_of(const GemmArgs& g, int blk) {
+  if (!g.sorted_ids) return 0;
+  const int e = g.block_expert[blk];
+  if (e < 0 || e >= g.E) {
+    set_device_error(kErrBlockExpert);
+    return 0;
+  }
+  return e;
 }
 
 // Bounded wait that ignores the abort flag: used while unwinding, to let
@@ -412,20 +428,33 @@ __device__ void quantize_rows_grid(const GemmArgs& g, int rows) {
   }
 }
 
-template <int BN, int STAGES, bool S1, int KIND>
+// PAIR = false: one CTA per tile (MMA M = 128). PAIR = true: a 2-CTA cluster
+// per tile of 256 weight rows (rank r holds weight sub-tile 2 * wt + r, the
+// sub-tile index the epilogue, the scale tiles and the fp8 partials use);
+// rank 0 issues the M = 256 MMAs; each rank loads its 128 weight rows and
+// half of the tile's token rows (split at ncols / 2), plus, for MX, its own
+// A scale tile and the whole B scale tile. Stage pipeline: each rank waits on
+// its own `empty` barriers; every load completes on rank 0's `full` barrier,
+// armed by rank 0 with the bytes of both; the MMA commits to `empty` and
+// `acc_full` of both ranks; every epilogue warp of both ranks arrives on rank
+// 0's `acc_empty`.
+template <int BN, int STAGES, bool S1, int KIND, bool PAIR = false>
 __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     k_moe_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmB16, const GemmArgs g) {
-  using L = GemmSmem<BN, STAGES, KIND, S1>;
+               const __grid_constant__ CUtensorMap tmB16, const __grid_constant__ CUtensorMap tmSfa,
+               const __grid_constant__ CUtensorMap tmSfb, const GemmArgs g) {
+  using L = GemmSmem<BN, STAGES, KIND, S1, PAIR>;
   constexpr bool FP8 = KIND == kFp8;
   constexpr bool MX = is_mx(KIND);
   constexpr int G = L::kGroups;
   constexpr int NACC = L::kAcc;
   constexpr int KE = KIND == kBf16 ? 64 : 128;  // K elements per stage
   constexpr int kUmmaKBytes = 32;               // K bytes per MMA: 16 bf16 or 32 e4m3
+  constexpr int kMmaM = PAIR ? 2 * kTileM : kTileM;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
   static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
+  static_assert(!PAIR || !(FP8 && S1), "fp8 stage 1 quantises h after a grid barrier: one CTA per tile");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -440,6 +469,10 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  // epilogue arrivals per accumulator phase: every thread (one CTA) or every
+  // epilogue warp of both CTAs (pair)
+  constexpr uint32_t kAccEmptyCount = PAIR ? 2 * (kEpiThreads / 32) : kEpiThreads;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -448,24 +481,46 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     }
     for (int a = 0; a < NACC; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], kEpiThreads);
+      mbar_init(&acc_empty[a], kAccEmptyCount);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, L::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, L::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // shared::cluster addresses of rank 0's full / acc_empty barriers and of
+  // both ranks' empty / acc_full barriers (pair only)
+  uint32_t full0 = 0, acc_empty0 = 0, empty_r[2] = {0, 0}, acc_full_r[2] = {0, 0};
+  if constexpr (PAIR) {
+    full0 = mapa_shared(smem_u32(full), 0);
+    acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
+    empty_r[0] = mapa_shared(smem_u32(empty), 0);
+    empty_r[1] = mapa_shared(smem_u32(empty), 1);
+    acc_full_r[0] = mapa_shared(smem_u32(acc_full), 0);
+    acc_full_r[1] = mapa_shared(smem_u32(acc_full), 1);
+  }
+
   int n_blocks = g.sorted_ids ? (*g.num_padded) / BN : g.identity_rows / BN;
   if (n_blocks > g.cap_blocks) n_blocks = g.cap_blocks;
-  const int total = n_blocks * g.n_mt;
+  // scheduling unit: one CTA (tile of 128 weight rows) or one pair (256 rows)
+  const int n_wt = PAIR ? g.n_mt / 2 : g.n_mt;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int total = n_blocks * n_wt;
   const int slots = g.T * g.top_k;
 
   if (warp == 0) {
@@ -476,11 +531,13 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     uint32_t phase = 0;
     uint32_t pending = 0, pend_parity = 0;  // stages armed and not yet re-acquired
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const int blk = tile / g.n_mt;
-      const int mt = tile - blk * g.n_mt;
-      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+    for (int tile = unit0; tile < total && ok; tile += n_units) {
+      const int blk = tile / n_wt;
+      const int mt = PAIR ? 2 * (tile - blk * n_wt) + static_cast<int>(rank) : tile - blk * n_wt;
+      const int expert = block_expert_of(g, blk);
       const int ncols = block_cols<BN>(g, blk, lane);  // token rows this tile loads and multiplies
+      const int my_rows = PAIR ? ncols / 2 : ncols;    // token rows this CTA loads
+      const int row0 = blk * BN + (PAIR ? static_cast<int>(rank) * my_rows : 0);
       for (int kb = 0; kb < g.num_kb; ++kb) {
         uint8_t* a_dst = smem + stage * L::kStageBytes;
         uint8_t* b_dst = a_dst + L::kABytes;
@@ -489,32 +546,56 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
         if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        if (lane == 0) {
-          pending &= ~(1u << stage);
-          // transaction bytes count what the copies read from global memory:
-          // half the shared-memory footprint for the packed e2m1 weight tile
-          uint32_t bytes = (KIND == kMx4 ? L::kABytes / 2 : L::kABytes) + static_cast<uint32_t>(ncols) * kTileKBytes;
-          if (MX) bytes += 2 * kSfTile;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
-          else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
-          // token rows as one box when the tile is full (B from x, the sorted copy, or h)
-          if (ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
-          if (MX) {
-            const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
-            bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
-            bulk_load(sfb_dst, (S1 ? g.xsf : g.hsf) + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile,
-                      kSfTile, &full[stage], pol_x);
+        // transaction bytes count what the copies read from global memory:
+        // half the shared-memory footprint for the packed e2m1 weight tile
+        uint32_t bytes = (KIND == kMx4 ? L::kABytes / 2 : L::kABytes) + static_cast<uint32_t>(my_rows) * kTileKBytes;
+        if (MX) bytes += 2 * kSfTile;
+        if constexpr (PAIR) {
+          const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
+          if (lane == 0) {
+            pending &= ~(1u << stage);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);  // both CTAs' copies
+            if (S1) tma_load_5d_pair(a_dst, &tmA, fb, kb * KE, 0, 0, mt * 4, expert, pol_w);
+            else tma_load_3d_pair(a_dst, &tmA, fb, kb * KE, mt * kTileM, expert, pol_w);
+            if (ncols == BN) tma_load_2d_pair(b_dst, &tmB, fb, kb * KE, row0, pol_x);
+            if (MX) {
+              const int wt = (expert * g.n_mt + mt) * g.num_kb + kb;
+              tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, wt * 32, pol_w);
+              tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 32, pol_x);
+            }
+            pending |= 1u << stage;
+            pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           }
-          pending |= 1u << stage;
-          pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
-        }
-        __syncwarp();
-        // a short tile: its token rows in 16-row boxes, issued by the lanes of
-        // the warp (the barrier was armed above with the stage's full byte count)
-        if (ncols < BN) {
-          for (int q = lane; q < ncols / 16; q += 32)
-            tma_load_2d(b_dst + q * 16 * kTileKBytes, &tmB16, &full[stage], kb * KE, blk * BN + q * 16, pol_x);
+          __syncwarp();
+          // a short tile: this CTA's token rows in 8-row boxes, issued by the lanes
+          if (ncols < BN) {
+            for (int q = lane; q < my_rows / 8; q += 32)
+              tma_load_2d_pair(b_dst + q * 8 * kTileKBytes, &tmB16, fb, kb * KE, row0 + q * 8, pol_x);
+          }
+        } else {
+          if (lane == 0) {
+            pending &= ~(1u << stage);
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+            else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
+            // token rows as one box when the tile is full (B from x, the sorted copy, or h)
+            if (ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+            if (MX) {
+              const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
+              bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
+              bulk_load(sfb_dst, (S1 ? g.xsf : g.hsf) + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile,
+                        kSfTile, &full[stage], pol_x);
+            }
+            pending |= 1u << stage;
+            pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+          }
+          __syncwarp();
+          // a short tile: its token rows in 16-row boxes, issued by the lanes of
+          // the warp (the barrier was armed above with the stage's full byte count)
+          if (ncols < BN) {
+            for (int q = lane; q < ncols / 16; q += 32)
+              tma_load_2d(b_dst + q * 16 * kTileKBytes, &tmB16, &full[stage], kb * KE, blk * BN + q * 16, pol_x);
+          }
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -524,21 +605,30 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
       __syncwarp();
     }
     if (!ok && lane == 0) {
-      for (int s = 0; s < STAGES; ++s)
-        if ((pending >> s) & 1u) drain_wait(&full[s], (pend_parity >> s) & 1u);
+      if (!PAIR || rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if ((pending >> s) & 1u) drain_wait(&full[s], (pend_parity >> s) & 1u);
+      } else if (pending) {
+        // rank 1's copies complete on rank 0's barriers, which it cannot wait
+        // on: give copies in flight a bounded 2 ms to land before unwinding
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) __nanosleep(1000);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // (a pair's MMAs are all issued by rank 0)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     uint32_t sf_slot = 0;
     int j = 0;  // local tile counter: accumulator j % NACC, use (j / NACC)
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+    const bool issuer = !PAIR || rank == 0;
+    for (int tile = unit0; issuer && tile < total; tile += n_units, ++j) {
       const int acc = j % NACC;
       const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
-      const int ncols = block_cols<BN>(g, tile / g.n_mt, lane);
-      const uint32_t idesc = FP8 ? idesc_e4m3(kTileM, ncols) : idesc_bf16(kTileM, ncols);
+      const int ncols = block_cols<BN>(g, tile / n_wt, lane);
+      const uint32_t idesc = FP8 ? idesc_e4m3(kMmaM, ncols) : idesc_bf16(kMmaM, ncols);
       if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -559,8 +649,13 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
             tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol) + sf_slot * 8;
             tsfb = tsfa + 4;
             const uint32_t sf_addr = a_addr + L::kABytes + L::kBBytes;
-            tmem_cp_32x128b_x4(tsfa, plain_rows16_desc(sf_addr));
-            tmem_cp_32x128b_x4(tsfb, plain_rows16_desc(sf_addr + kSfTile));
+            if constexpr (PAIR) {
+              tmem_cp_32x128b_x4_pair(tsfa, plain_rows16_desc(sf_addr));
+              tmem_cp_32x128b_x4_pair(tsfb, plain_rows16_desc(sf_addr + kSfTile));
+            } else {
+              tmem_cp_32x128b_x4(tsfa, plain_rows16_desc(sf_addr));
+              tmem_cp_32x128b_x4(tsfb, plain_rows16_desc(sf_addr + kSfTile));
+            }
             sf_slot = (sf_slot + 1) % kSfSlots;
           }
 #pragma unroll
@@ -571,14 +666,24 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
             if (MX) {
               // K block kk of the stage: byte kk of each scale column
               const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-              umma_mx8(d_tmem, adesc + adv, bdesc + adv, idesc_mx(kTileM, ncols, kk, KIND == kMx4 ? kFmtE2M1 : kFmtE4M3), tsfa | sel, tsfb | sel, accum);
+              const uint32_t id = idesc_mx(kMmaM, ncols, kk, KIND == kMx4 ? kFmtE2M1 : kFmtE4M3);
+              if constexpr (PAIR) umma_mx8_pair(d_tmem, adesc + adv, bdesc + adv, id, tsfa | sel, tsfb | sel, accum);
+              else umma_mx8(d_tmem, adesc + adv, bdesc + adv, id, tsfa | sel, tsfb | sel, accum);
             } else if (FP8) {
-              umma_f8(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
+              if constexpr (PAIR) umma_f8_pair(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
+              else umma_f8(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
             } else {
-              umma_f16(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
+              if constexpr (PAIR) umma_f16_pair(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
+              else umma_f16(d_tmem, adesc + adv, bdesc + adv, idesc, accum);
             }
           }
-          umma_commit(&empty[stage]);  // smem stage free once these MMAs (and copies) finish
+          // smem stage free once these MMAs (and copies) finish: in both CTAs for a pair
+          if constexpr (PAIR) {
+            umma_commit_pair(empty_r[0] + 8u * static_cast<uint32_t>(stage));
+            umma_commit_pair(empty_r[1] + 8u * static_cast<uint32_t>(stage));
+          } else {
+            umma_commit(&empty[stage]);
+          }
         }
         __syncwarp();
         if (++stage == STAGES) {
@@ -587,11 +692,19 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
         }
       }
       if (!ok) break;
-      if (lane == 0) umma_commit(&acc_full[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR) {
+          umma_commit_pair(acc_full_r[0] + 8u * static_cast<uint32_t>(acc));
+          umma_commit_pair(acc_full_r[1] + 8u * static_cast<uint32_t>(acc));
+        } else {
+          umma_commit(&acc_full[acc]);
+        }
+      }
       __syncwarp();
     }
     if (!ok && lane == 0) {
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair(mapa_shared(smem_u32(drain), 0));
+      else umma_commit(drain);
       drain_wait(drain, 0);
     }
   } else {
@@ -607,14 +720,25 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
                                                             // stage 2 top-k weight (x h and W2 scales for fp8)
     int* last_sm = reinterpret_cast<int*>(wgt_sm + BN);
     float* amax_part = reinterpret_cast<float*>(last_sm + BN);
+    // the accumulator is free again once this thread's (one CTA) or this
+    // warp's (pair: every warp of both CTAs arrives on rank 0) reads are done
+    auto release_acc = [&](int acc) {
+      tc_fence_before();
+      if constexpr (PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(acc));
+      } else {
+        mbar_arrive(&acc_empty[acc]);
+      }
+    };
     int j = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+    for (int tile = unit0; tile < total; tile += n_units, ++j) {
       if (j % G != grp) continue;
-      const int blk = tile / g.n_mt;
-      const int mt = tile - blk * g.n_mt;
+      const int blk = tile / n_wt;
+      const int mt = PAIR ? 2 * (tile - blk * n_wt) + static_cast<int>(rank) : tile - blk * n_wt;
       const int acc = j % NACC;
       const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
-      const int expert = g.sorted_ids ? g.block_expert[blk] : 0;
+      const int expert = block_expert_of(g, blk);
       const int ncols = block_cols<BN>(g, blk, lane);  // accumulator columns the MMA wrote
 
       // per-column metadata, fetched while the accumulator is still being built
@@ -655,10 +779,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           float v[16];
           tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
           tmem_wait_ld();
-          if (c0 + 16 >= ncols) {
-            tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
-          }
+          if (c0 + 16 >= ncols) release_acc(acc);
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
             const float o0 = __shfl_xor_sync(0xffffffffu, v[i], 16);
@@ -744,10 +865,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           float v[16];
           tmem_ld16(t_row + static_cast<uint32_t>(c0), v);
           tmem_wait_ld();
-          if (c0 + 16 >= ncols) {
-            tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
-          }
+          if (c0 + 16 >= ncols) release_acc(acc);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int t = tok_sm[c0 + i];
@@ -839,9 +957,11 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, L::kTmemCols);
+    else tmem_dealloc(tmem_base, L::kTmemCols);
   }
   if constexpr (FP8 && S1) {
     if (g.quant_phase && grid_barrier(g.grid_bar, reinterpret_cast<int*>(tmem_slot + 2)))

@@ -6,6 +6,7 @@
 // below and are compiled into this one translation unit.
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -96,6 +97,15 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
   return MOE_OK;
 }
 
+// Map of an MX scale-tile array (512-byte tiles) as rows of 16 bytes: one
+// 16 x 32 box is one tile, landing dense in shared memory (no swizzle).
+moe_status_t make_sf_tile_map(CUtensorMap* m, const void* base, size_t tiles) {
+  const cuuint64_t dims[2] = {16, static_cast<cuuint64_t>(tiles) * 32};
+  const cuuint64_t st[1] = {16};
+  const cuuint32_t box[2] = {16, 32};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 // ------------------------------------------------------------ GEMM dispatch
 
 template <int BN, int KIND>
@@ -109,31 +119,112 @@ constexpr int stages_for() {
   return BN == 16 ? 6 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
 }
 
+// Pair tiles: as many stages as fit in 227 KB (each CTA holds half the token rows).
+template <int BN, int KIND, bool S1, int ST = 2>
+constexpr int pair_stages() {
+  if constexpr (ST < 16 && moe::GemmSmem<BN, ST + 1, KIND, S1, true>::kBytes <= 227 * 1024)
+    return pair_stages<BN, KIND, S1, ST + 1>();
+  else
+    return ST;
+}
+
+// Whether a GEMM runs on CTA pairs (one MMA of M = 256 per pair, each SM
+// loading its 128 weight rows and half the token tile): 128-token tiles, an
+// even number of 128-row weight sub-tiles, not the fp8 stage 1 (its per-row
+// quantisation of h follows a grid barrier in a cooperative launch). At
+// 128-token tiles the kernels are paced by the operand bytes each SM brings
+// into shared memory, and a pair brings 24 KB + scales per stage for what one
+// CTA needed 32 KB. MOE_B200_PAIR=0 in the environment selects single CTAs
+// everywhere (same results).
+bool use_pair(int dtype, int bm, int n_mt, bool s1) {
+  static const bool enabled = [] {
+    const char* v = getenv("MOE_B200_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return enabled && bm == 128 && n_mt % 2 == 0 && !(s1 && dtype == MOE_DT_FP8_E4M3);
+}
+
+template <typename Kern>
+moe_status_t set_smem_attr(Kern kern, int bytes, std::atomic<int>* attr_set) {
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load()) {
+    MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+  }
+  return MOE_OK;
+}
+
 template <int BN, bool S1, int KIND>
 moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb16,
                             const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
   constexpr int ST = stages_for<BN, KIND>();
   using L = moe::GemmSmem<BN, ST, KIND, S1>;
   static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
-  auto kern = moe::k_moe_gemm<BN, ST, S1, KIND>;
+  auto kern = moe::k_moe_gemm<BN, ST, S1, KIND, false>;
   static std::atomic<int> attr_set[64];
-  int dev = 0;
-  MOE_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64 || !attr_set[dev].load()) {
-    MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
-    if (dev >= 0 && dev < 64) attr_set[dev].store(1);
-  }
+  const moe_status_t r = set_smem_attr(kern, L::kBytes, attr_set);
+  if (r != MOE_OK) return r;
   int grid = max_tiles < num_sms() ? max_tiles : num_sms();
   if (grid < 1) grid = 1;
+  // the scale-tile maps are read by pair kernels only
   if (g.quant_phase) {
     // every CTA resident at once (one per SM): the grid barrier's wait ends
     void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<CUtensorMap*>(&tb16),
-                    const_cast<moe::GemmArgs*>(&g)};
+                    const_cast<CUtensorMap*>(&tb), const_cast<CUtensorMap*>(&tb), const_cast<moe::GemmArgs*>(&g)};
     MOE_CK(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid),
                                        dim3(moe::EpiCfg<BN, KIND, S1>::kThreads), args, L::kBytes, s));
   } else {
-    kern<<<grid, moe::EpiCfg<BN, KIND, S1>::kThreads, L::kBytes, s>>>(ta, tb, tb16, g);
+    kern<<<grid, moe::EpiCfg<BN, KIND, S1>::kThreads, L::kBytes, s>>>(ta, tb, tb16, tb, tb, g);
   }
+  MOE_CK(cudaGetLastError());
+  return MOE_OK;
+}
+
+// A GEMM on CTA pairs: 2-CTA clusters, as many as can be resident at once
+// (cudaOccupancyMaxActiveClusters), each looping over pair tiles.
+template <bool S1, int KIND>
+moe_status_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb8,
+                              const CUtensorMap& tsfa, const CUtensorMap& tsfb, const moe::GemmArgs& g,
+                              int max_pair_tiles, cudaStream_t s) {
+  constexpr int BN = 128;
+  constexpr int ST = pair_stages<BN, KIND, S1>();
+  using L = moe::GemmSmem<BN, ST, KIND, S1, true>;
+  static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
+  auto kern = moe::k_moe_gemm<BN, ST, S1, KIND, true>;
+  constexpr int threads = moe::EpiCfg<BN, KIND, S1>::kThreads;
+  static std::atomic<int> attr_set[64];
+  moe_status_t r = set_smem_attr(kern, L::kBytes, attr_set);
+  if (r != MOE_OK) return r;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  static std::atomic<int> max_clusters[64];
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  int mc = (dev >= 0 && dev < 64) ? max_clusters[dev].load() : 0;
+  if (mc == 0) {
+    cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1));
+    if (cudaOccupancyMaxActiveClusters(&mc, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess || mc < 1) {
+      cudaGetLastError();  // clear: fall back to one pair per two SMs
+      mc = num_sms() / 2;
+    }
+    if (dev >= 0 && dev < 64) max_clusters[dev].store(mc);
+  }
+  int clusters = max_pair_tiles < mc ? max_pair_tiles : mc;
+  if (clusters < 1) clusters = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+  void* args[] = {const_cast<CUtensorMap*>(&ta), const_cast<CUtensorMap*>(&tb), const_cast<CUtensorMap*>(&tb8),
+                  const_cast<CUtensorMap*>(&tsfa), const_cast<CUtensorMap*>(&tsfb), const_cast<moe::GemmArgs*>(&g)};
+  MOE_CK(cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(kern), args));
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }
@@ -160,6 +251,19 @@ moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CU
   if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm<S1, moe::kMx8>(bm, ta, tb, tb16, g, max_tiles, s);
   if (dtype == MOE_DT_MXFP4_E2M1) return launch_gemm<S1, moe::kMx4>(bm, ta, tb, tb16, g, max_tiles, s);
   return launch_gemm<S1, moe::kBf16>(bm, ta, tb, tb16, g, max_tiles, s);
+}
+
+template <bool S1>
+moe_status_t launch_gemm_pair_kind(int dtype, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb8,
+                                   const CUtensorMap& tsfa, const CUtensorMap& tsfb, const moe::GemmArgs& g,
+                                   int max_pair_tiles, cudaStream_t s) {
+  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm_pair<S1, moe::kMx8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  if (dtype == MOE_DT_MXFP4_E2M1) return launch_gemm_pair<S1, moe::kMx4>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  if constexpr (!S1) {
+    if (dtype == MOE_DT_FP8_E4M3) return launch_gemm_pair<S1, moe::kFp8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  }
+  if (dtype == MOE_DT_BF16) return launch_gemm_pair<S1, moe::kBf16>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  return MOE_ERR_INVALID_ARG;
 }
 
 // Padded sorted length bound T*k + E*(bm-1), rounded up to whole blocks.
@@ -273,6 +377,34 @@ moe_status_t launch_router_gemm_vpl(const moe::RouterGemmArgs& a, cudaStream_t s
   if (vpl <= 4) return wide ? launch_router_gemm<4, 16, TX>(a, s) : launch_router_gemm<4, 4, TX>(a, s);
   if (vpl <= 8) return wide ? launch_router_gemm<8, 16, TX>(a, s) : launch_router_gemm<8, 4, TX>(a, s);
   return launch_router_gemm<16, 4, TX>(a, s);
+}
+
+// Argument checks of stage 2, shared by moe_stage2_gemm_accumulate and
+// moe_stage2_gemm_accumulate_static_ws so that both accept and refuse the same
+// calls, before anything is enqueued (the workspace is checked by each).
+moe_status_t check_stage2(int dtype, const void* h, const void* h_scale, const void* w2, const void* w2_scale,
+                          const void* weights, int weights_dtype, const int32_t* sorted_ids,
+                          const int32_t* block_expert, const int32_t* num_padded, int T, int top_k, int H, int I,
+                          int E, int block_m, const void* addend, const void* out) {
+  const bool fp8 = dtype == MOE_DT_FP8_E4M3;
+  const bool mx = is_mx_dtype(dtype);
+  const bool w4 = dtype == MOE_DT_MXFP4_E2M1;
+  if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
+    return MOE_ERR_INVALID_ARG;
+  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
+  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
+  if ((fp8 || mx) && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (mx && block_m > 128) return MOE_ERR_INVALID_ARG;
+  if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
+    return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
+  if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;
+  if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)) ||
+      (mx && (!aligned16(h_scale) || !aligned16(w2_scale))) || (w4 && !aligned32(w2)))
+    return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
 }
 
 extern "C" {
@@ -487,7 +619,8 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint8_t* xs = permute ? wsb + L.xs_off : nullptr;
   uint8_t* xsf = mx ? wsb + L.xsf_off : nullptr;
-  CUtensorMap ta, tb, tb16;
+  const bool pair = use_pair(dtype, block_m, I / 64, true);
+  CUtensorMap ta, tb, tb16, tsfa, tsfb;
   {
     // MXFP4: dims count e2m1 elements, strides bytes (two elements a byte);
     // the 16U4_ALIGN16B type spreads each 8 bytes over 16 in shared memory
@@ -502,17 +635,29 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   {
     // token rows: one [block_m x 128 B] box per stage from the sorted copy,
     // or from x itself with identity routing (rows past T read as zeros);
-    // tb16: the same rows in 16-row boxes, for tiles with fewer token rows
+    // tb16: the same rows in 16-row boxes, for tiles with fewer token rows.
+    // A CTA pair splits the token rows: boxes of block_m / 2 rows, and 8-row
+    // boxes for short tiles.
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), permute ? static_cast<cuuint64_t>(rows_cap)
                                                                     : static_cast<cuuint64_t>(T)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(H) * es};
     const void* base = permute ? static_cast<const void*>(xs) : x;
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(pair ? block_m / 2 : block_m)};
     moe_status_t r = make_map(&tb, tdt, 2, base, dims, st, box);
     if (r != MOE_OK) return r;
-    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
+    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), pair ? 8u : 16u};
     r = make_map(&tb16, tdt, 2, base, dims, st, box16);
     if (r != MOE_OK) return r;
+  }
+  if (pair && mx) {
+    // pairs load the scale tiles by TMA (their copies complete on rank 0's barrier)
+    moe_status_t r = make_sf_tile_map(&tsfa, w13_scale, static_cast<size_t>(E) * (I / 64) * (H / 128));
+    if (r != MOE_OK) return r;
+    r = make_sf_tile_map(&tsfb, xsf, static_cast<size_t>(cap_blocks) * (H / 128));
+    if (r != MOE_OK) return r;
+  } else {
+    tsfa = tb;  // not read
+    tsfb = tb;
   }
   moe::GemmArgs g{};
   g.sorted_ids = sorted_ids;
@@ -524,6 +669,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
   g.top_k = top_k;
   g.H = H;
   g.I = I;
+  g.E = E;
   g.n_mt = I / 64;
   g.num_kb = H / ke;
   g.rows_cap = static_cast<int>(rows_cap);
@@ -569,6 +715,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     MOE_CK(cudaGetLastError());
   }
   const int max_tiles = cap_blocks * g.n_mt;
+  if (pair) return launch_gemm_pair_kind<true>(dtype, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
   return launch_gemm_kind<true>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
@@ -578,26 +725,14 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
                                         const int32_t* num_padded, int T, int top_k, int H, int I, int E,
                                         int block_m, const void* addend, moe_event_t addend_ready, void* acc_ws,
                                         void* out, moe_stream_t stream) {
+  const moe_status_t chk = check_stage2(dtype, h, h_scale, w2, w2_scale, weights, weights_dtype, sorted_ids,
+                                        block_expert, num_padded, T, top_k, H, I, E, block_m, addend, out);
+  if (chk != MOE_OK) return chk;
+  if (top_k > 1 && !acc_ws) return MOE_ERR_INVALID_ARG;
+  if (acc_ws && !aligned16(acc_ws)) return MOE_ERR_ALIGNMENT;
   const bool fp8 = dtype == MOE_DT_FP8_E4M3;
   const bool mx = is_mx_dtype(dtype);
   const bool w4 = dtype == MOE_DT_MXFP4_E2M1;
-  if (dtype != MOE_DT_BF16 && !fp8 && !mx) return MOE_ERR_UNSUPPORTED_DTYPE;
-  if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
-  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
-    return MOE_ERR_INVALID_ARG;
-  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
-  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  if (top_k > 1 && !acc_ws) return MOE_ERR_INVALID_ARG;
-  if ((fp8 || mx) && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
-  if (mx && block_m > 128) return MOE_ERR_INVALID_ARG;
-  if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
-    return MOE_ERR_UNSUPPORTED_DTYPE;
-  if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
-  if (mx && I % 128 != 0) return MOE_ERR_ALIGNMENT;
-  if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)) ||
-      (acc_ws && !aligned16(acc_ws)) || (mx && (!aligned16(h_scale) || !aligned16(w2_scale))) ||
-      (w4 && !aligned32(w2)))
-    return MOE_ERR_ALIGNMENT;
 
   const bool b16 = dtype == MOE_DT_BF16;
   const int es = b16 ? 2 : 1;
@@ -606,7 +741,8 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   // identity routing launches over the blocks that hold tokens only
   const int cap_blocks = sorted_ids ? static_cast<int>(rows_cap / block_m) : (T + block_m - 1) / block_m;
   const CUtensorMapDataType tdt = b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  CUtensorMap ta, tb, tb16;
+  const bool pair = use_pair(dtype, block_m, H / moe::kTileM, false);
+  CUtensorMap ta, tb, tb16, tsfa, tsfb;
   {
     const size_t wrow = w4 ? static_cast<size_t>(I) / 2 : static_cast<size_t>(I) * es;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(H),
@@ -619,12 +755,21 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(rows_cap)};
     const cuuint64_t st[1] = {static_cast<cuuint64_t>(I) * es};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(block_m)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ke), static_cast<cuuint32_t>(pair ? block_m / 2 : block_m)};
     moe_status_t r = make_map(&tb, tdt, 2, h, dims, st, box);
     if (r != MOE_OK) return r;
-    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), 16};
+    const cuuint32_t box16[2] = {static_cast<cuuint32_t>(ke), pair ? 8u : 16u};
     r = make_map(&tb16, tdt, 2, h, dims, st, box16);
     if (r != MOE_OK) return r;
+  }
+  if (pair && mx) {
+    moe_status_t r = make_sf_tile_map(&tsfa, w2_scale, static_cast<size_t>(E) * (H / 128) * (I / 128));
+    if (r != MOE_OK) return r;
+    r = make_sf_tile_map(&tsfb, h_scale, static_cast<size_t>(cap_blocks) * (I / 128));
+    if (r != MOE_OK) return r;
+  } else {
+    tsfa = tb;  // not read
+    tsfb = tb;
   }
   cudaStream_t s = as_stream(stream);
   if (addend_ready) MOE_CK(cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(addend_ready), 0));
@@ -639,6 +784,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.top_k = top_k;
   g.H = H;
   g.I = I;
+  g.E = E;
   g.n_mt = H / moe::kTileM;
   g.num_kb = (I + ke - 1) / ke;
   g.rows_cap = static_cast<int>(rows_cap);
@@ -656,6 +802,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
+  if (pair) return launch_gemm_pair_kind<false>(dtype, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
   return launch_gemm_kind<false>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
@@ -691,21 +838,11 @@ moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, cons
                                                   const int32_t* num_padded, int T, int top_k, int H, int I, int E,
                                                   int block_m, const void* addend, moe_event_t addend_ready,
                                                   void* out, moe_stream_t stream) {
-  // The argument checks of moe_stage2_gemm_accumulate, repeated here so that
-  // nothing (not even the clearing memset) is enqueued for an invalid call.
-  if (dtype != MOE_DT_BF16 && dtype != MOE_DT_FP8_E4M3 && !is_mx_dtype(dtype)) return MOE_ERR_UNSUPPORTED_DTYPE;
-  if (!h || !w2 || !out) return MOE_ERR_INVALID_ARG;
-  if (T < 1 || top_k < 1 || E < 1 || top_k > E || H < 1 || I < 1 || !valid_block_m(block_m))
-    return MOE_ERR_INVALID_ARG;
-  if (sorted_ids && (!block_expert || !num_padded)) return MOE_ERR_INVALID_ARG;
-  if (!sorted_ids && top_k != 1) return MOE_ERR_INVALID_ARG;
-  if (dtype != MOE_DT_BF16 && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
-  if (is_mx_dtype(dtype) && (block_m > 128 || I % 128 != 0)) return MOE_ERR_INVALID_ARG;
-  if (weights && weights_dtype != MOE_DT_F32 && weights_dtype != MOE_DT_BF16 && weights_dtype != MOE_DT_FP16)
-    return MOE_ERR_UNSUPPORTED_DTYPE;
-  if (H % 128 != 0 || I % 64 != 0) return MOE_ERR_SHAPE;
-  if (!aligned16(h) || !aligned16(w2) || !aligned16(out) || (addend && !aligned16(addend)))
-    return MOE_ERR_ALIGNMENT;
+  // the checks of moe_stage2_gemm_accumulate first: nothing (not even the
+  // clearing memset) is enqueued for a call that one of them refuses
+  const moe_status_t chk = check_stage2(dtype, h, h_scale, w2, w2_scale, weights, weights_dtype, sorted_ids,
+                                        block_expert, num_padded, T, top_k, H, I, E, block_m, addend, out);
+  if (chk != MOE_OK) return chk;
   void* ws = nullptr;
   if (top_k > 1) {
     const size_t need = moe_stage2_workspace_bytes(T, H);
@@ -714,6 +851,15 @@ moe_status_t moe_stage2_gemm_accumulate_static_ws(int dtype, const void* h, cons
                "stage-2 workspace of %zu bytes exceeds the static %u bytes (T=%d, H=%d)", need,
                static_cast<unsigned>(MOE_STAGE2_STATIC_WS_BYTES), T, H);
       return MOE_ERR_WORKSPACE_LIMIT;
+    }
+    // the array used is the current device's: the stream must belong to it
+    int dev = 0, sdev = 0;
+    MOE_CK(cudaGetDevice(&dev));
+    MOE_CK(cudaStreamGetDevice(as_stream(stream), &sdev));
+    if (sdev != dev) {
+      snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+               "stream of device %d while device %d is current", sdev, dev);
+      return MOE_ERR_DEVICE;
     }
     const moe_status_t r = static_ws_address(&ws);
     if (r != MOE_OK) return r;

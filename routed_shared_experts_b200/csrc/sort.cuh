@@ -1,4 +1,4 @@
-// sort.cuh - align/sort of the routed slots by expert, one CTA.
+// sort.cuh - align/sort of the routed slots by expert, one CTA of 32 warps.
 //
 // vllm-project/vllm PR 65207, reviewer measurements ("Commits 2 and 3"):
 // moe_sorting is run without zeroing the layer output; here the sort never
@@ -22,6 +22,19 @@ struct SortArgs {
 };
 
 // Shared memory: cnt[E], base[E], warp_cnt[32][E], warp totals [32].
+//
+// Each warp owns one contiguous chunk of the flat slots (warp w: chunk w of
+// 32), so that a stable order needs no barrier per round:
+//   1. each warp counts its chunk's slots per expert into its own row of
+//      warp_cnt (32 slots per step, __match_any_sync groups equal experts, the
+//      lowest lane of a group adds the group's size: one writer per entry);
+//   2. per expert, an exclusive prefix over the 32 warps' counts, and over
+//      the experts an exclusive prefix of the padded segment sizes, turn each
+//      warp_cnt entry into the absolute position of that warp's first slot of
+//      that expert; counts, offsets, block owners and padding are written;
+//   3. each warp walks its chunk again in order and places every slot at its
+//      entry plus its rank among the equal experts of its 32-slot step, then
+//      advances the entry: ascending f inside every expert segment.
 __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   extern __shared__ int ssm[];
   const int E = a.E;
@@ -32,22 +45,41 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  const int chunk = (a.N + 31) / 32;
+  const int f0 = warp * chunk;
+  const int f1 = f0 + chunk < a.N ? f0 + chunk : a.N;
+  int* my_cnt_row = warp_cnt + warp * E;
 
-  for (int e = tid; e < E; e += kSortThreads) cnt[e] = 0;
+  for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
   __syncthreads();
-  for (int f = tid; f < a.N; f += kSortThreads) {
-    const int e = a.ids[f];
-    if (e >= 0 && e < E) {
-      atomicAdd(&cnt[e], 1);
-    } else {
+
+  // 1. per-warp counts
+  for (int b = f0; b < f1; b += 32) {
+    const int f = b + lane;
+    int e = f < f1 ? a.ids[f] : -1;
+    if (e >= E || (f < f1 && e < 0)) {
       set_device_error(kErrExpertRange);
+      e = -1;
     }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0) my_cnt_row[e] += __popc(peers);
+    __syncwarp();  // this step's counts before the next step's reads
   }
   __syncthreads();
 
-  // Exclusive prefix sum of the padded segment sizes (E <= 1024: one per thread).
-  const int my_cnt = tid < E ? cnt[tid] : 0;
-  const int my_pad = (my_cnt + a.bm - 1) / a.bm * a.bm;
+  // 2. exclusive prefix over warps (per expert), then over padded segments
+  int my_cnt = 0;
+  if (tid < E) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = warp_cnt[w * E + tid];
+      warp_cnt[w * E + tid] = run;
+      run += c;
+    }
+    my_cnt = run;
+    cnt[tid] = run;
+  }
+  const int my_pad = tid < E ? (my_cnt + a.bm - 1) / a.bm * a.bm : 0;
   int incl = my_pad;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -78,33 +110,25 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
     }
     for (int b = excl / a.bm; b < (excl + my_pad) / a.bm; ++b) a.block_expert[b] = tid;
     for (int p = excl + my_cnt; p < excl + my_pad; ++p) a.sorted[p] = a.N;  // sentinel
+    for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += excl;  // absolute start of warp w's slots of tid
   }
   __syncthreads();
 
-  // Stable placement, 1024 slots per round: position = segment base + slots
-  // of the same expert in earlier warps of this round + rank inside the warp.
-  for (int start = 0; start < a.N; start += kSortThreads) {
-    const int f = start + tid;
-    int e = f < a.N ? a.ids[f] : -1;
+  // 3. stable placement, each warp in its chunk's order
+  for (int b = f0; b < f1; b += 32) {
+    const int f = b + lane;
+    int e = f < f1 ? a.ids[f] : -1;
     if (e >= E) e = -1;
-    for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
-    __syncthreads();
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && rank == 0) warp_cnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    if (tid < E) {
-      int run = base[tid];
-      for (int w = 0; w < 32; ++w) {
-        const int c = warp_cnt[w * E + tid];
-        warp_cnt[w * E + tid] = run;
-        run += c;
-      }
-      base[tid] = run;
+    const uint32_t lower = peers & ((1u << lane) - 1u);
+    int pos = 0;
+    if (e >= 0) pos = my_cnt_row[e] + __popc(lower);
+    __syncwarp();
+    if (e >= 0) {
+      a.sorted[pos] = f;
+      if (lower == 0) my_cnt_row[e] += __popc(peers);
     }
-    __syncthreads();
-    if (e >= 0) a.sorted[warp_cnt[warp * E + e] + rank] = f;
-    __syncthreads();
+    __syncwarp();
   }
 }
 
