@@ -5,31 +5,36 @@
     torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU)
 
 A step is one forward of the whole layer (router top-k, align/sort, stage 1,
-stage 2 with the fused epilogue, and the side-stream shared expert with its
-gate) over one batch of T tokens of the decode workload (T=32, H=2048, E=128,
-top_k=8, I=768, shared Is=512, bf16; synthetic seeded inputs and weights).
-The layer does not shard: under torchrun every rank runs its own replica on its
-own GPU (weak scaling) and only the barrier and the max-over-ranks timing cross
-ranks.
+stage 2 with the fused epilogue, and the side-stream shared expert) over one
+batch of T tokens. The headline workload is the MXFP8 prefill layer (T=4096,
+H=7168, E=256, top_k=8, I=2048, shared Is=2048, e4m3 with ue8m0 scales per 32
+K elements, grouped sigmoid routing with a Zipf logit bias); the bf16 decode
+layer (T=32, H=2048, E=128, top_k=8, I=768, Is=512, gated shared expert) is
+measured in the same run and reported under "extra". Inputs and weights are
+synthetic and seeded. The layer does not shard: under torchrun every rank runs
+its own replica on its own GPU (weak scaling) and only the barrier and the
+max-over-ranks timing cross ranks.
 
-Timed region: K steps replayed from CUDA graphs (both streams captured), with
-the weights already resident in device memory. No L2 flush is done: for the
-default workload the activated experts' weights (~0.8 GB per step) exceed the
-126 MB L2, so every step reads them from HBM; `config.l2` states how each
-workload's step bytes compare with the L2. The dominant kernel's duration is
-taken from timing events captured inside the graph on its own stream. One JSON
-line is printed by rank 0.
+Timed region: exactly K steps replayed from CUDA graphs (both streams
+captured), no timing events inside, inputs and weights resident in device
+memory. Steps that read less than 3x the 126 MB L2 cycle through enough
+independent weight copies that every step's weights come from HBM
+(`config.l2`, `config.weight_copies`). Kernel durations for the roofline come
+from the same graph with events around the two GEMMs, replayed once right
+after the timed region. One JSON line is printed by rank 0.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +45,8 @@ from routed_shared_experts_b200 import configs, synth  # noqa: E402
 
 METRIC = "MoE layer tokens/s"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "decode_bf16"
+DEFAULT_WORKLOAD = "mxfp8_prefill"
+EXTRA_WORKLOADS = "decode_bf16"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
@@ -48,13 +54,19 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_WORKLOAD)
     ap.add_argument("--unroll", type=int, default=20, help="steps per captured graph")
-    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--extra", default=EXTRA_WORKLOADS,
+                    help="comma-separated workloads measured after the headline and reported under 'extra' "
+                         "('none' to skip)")
+    ap.add_argument("--extra-min-steps", type=int, default=2000, help="at least this many steps per extra workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="mark the timed region with the NVTX range 'moe_steady_state' (for a launch list of it)")
     ap.add_argument("--router-gemm", action="store_true",
                     help="start each step from the router linear x . W_r (moe_router_gemm_topk) instead of logits")
     ap.add_argument("--fused-shared", action="store_true",
@@ -200,16 +212,12 @@ def max_over_ranks(v: float, world: int) -> float:
 L2_BYTES = 126e6
 
 
-def l2_note(step_bytes: float) -> str:
-    """How the step's bytes relate to the 126 MB L2 between timed steps (no
-    flush is done; the weights are not cycled through copies)."""
-    if step_bytes >= 3 * L2_BYTES:
-        return f"no flush: the step reads {step_bytes / 1e9:.2f} GB, over 3x the 126 MB L2, so weights come from HBM"
-    if step_bytes > L2_BYTES:
-        return (f"no flush: the step reads {step_bytes / 1e6:.0f} MB, 1-3x the 126 MB L2; part of the weights "
-                "may still be in L2 from the previous step")
-    return (f"no flush: the step reads {step_bytes / 1e6:.1f} MB, under the 126 MB L2, so the weights stay "
-            "L2-resident across steps (launch-bound case, HBM roofline not meaningful)")
+def l2_note(step_bytes: float, copies: int = 1) -> str:
+    """How the step's bytes relate to the 126 MB L2 between timed steps."""
+    if copies > 1:
+        return (f"HBM: the step reads {step_bytes / 1e6:.1f} MB; steps cycle through {copies} weight copies "
+                f"({copies * step_bytes / 1e6:.0f} MB, over 3x the 126 MB L2), so each step's weights come from HBM")
+    return f"HBM: the step reads {step_bytes / 1e9:.2f} GB, over 3x the 126 MB L2, so weights come from HBM (no flush needed)"
 
 
 def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
@@ -256,95 +264,120 @@ def algorithmic_bytes(cfg, counts, router_gemm=False, quantize_x=False):
 # ----------------------------------------------------------------- our arm
 
 
-def run_ours(args):
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
+def weight_copies(step_bytes: float) -> int:
+    """Independent weight copies a run cycles through so that each step reads
+    its weights from HBM: enough copies that consecutive uses of one copy are
+    over 3x the L2 apart (the rotating-copies method of vllm-project/vllm PR
+    65207, reviewer measurements "Commit 1": 12 layers cycling 6 weight
+    copies)."""
+    return max(1, math.ceil(3 * L2_BYTES / max(step_bytes, 1.0)))
 
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    from routed_shared_experts_b200 import capi
+WEIGHT_KEYS = ("w13", "w2", "w13s", "w2s", "w13_scale", "w2_scale", "w13s_scale", "w2s_scale", "w_gate")
+
+
+def build_layers(cfg, inp, args, copies):
+    """The layer and copies - 1 more whose weights are clones (activations
+    and routing inputs shared, so every copy computes the same step)."""
     from routed_shared_experts_b200.layer import FusedSharedMoELayer, MoELayer
+
+    def make(d):
+        if args.fused_shared:
+            return FusedSharedMoELayer(cfg, d)
+        return MoELayer(cfg, d, router_gemm=args.router_gemm, quantize_x=args.quantize_x)
+    layers = [make(inp)]
+    for _ in range(copies - 1):
+        d = dict(inp)
+        for k in WEIGHT_KEYS:
+            if d.get(k) is not None:
+                d[k] = d[k].clone()
+        layers.append(make(d))
+    return layers
+
+
+def measure(cfg, args, dev, world, steps, warmup, e2e_steps, clocks_local):
+    """One workload: warm-up, then exactly `steps` steps replayed from CUDA
+    graphs with no timing events inside (max over ranks), then the same graph
+    shape with per-kernel timing events replayed once more for kernel
+    durations, then the e2e serving loop with host buffers."""
+    from routed_shared_experts_b200 import capi
     from routed_shared_experts_b200.pipeline import StepPipeline
 
-    cfg = configs.CONFIGS[args.config]
     inp = synth.make_layer_inputs(cfg, device=dev)
     if args.router_gemm and cfg.dtype == "bf16":
         inp["x_r"] = inp["x"]  # the same bf16 activations feed the router linear and stage 1
-    if args.fused_shared:
-        if args.router_gemm or args.quantize_x:
-            raise SystemExit("--fused-shared runs from logits and pre-quantised x")
-        layer = FusedSharedMoELayer(cfg, inp)
-    else:
-        layer = MoELayer(cfg, inp, router_gemm=args.router_gemm, quantize_x=args.quantize_x)
+    if args.fused_shared and (args.router_gemm or args.quantize_x):
+        raise SystemExit("--fused-shared runs from logits and pre-quantised x")
     main = torch.cuda.Stream(device=dev)
+    first = build_layers(cfg, inp, args, 1)[0]
     with torch.cuda.stream(main):
-        layer.forward(main)
+        first.forward(main)
     torch.cuda.synchronize()
     if capi.device_error(main) != 0:
         raise RuntimeError("device error after the first step")
-    counts = layer.expert_counts.cpu()[: cfg.E]  # routed experts (the fused layer appends the shared pieces)
+    counts = first.expert_counts.cpu()[: cfg.E]  # routed experts (the fused layer appends the shared pieces)
     ab = algorithmic_bytes(cfg, counts, args.router_gemm, args.quantize_x)
+    copies = weight_copies(ab["layer"])
+    layers = [first] + (build_layers(cfg, inp, args, copies)[1:] if copies > 1 else [])
 
-    # graphs: U unrolled plain steps, the same U steps with timing events
-    # around the two GEMMs (events inside a graph add a few microseconds each,
-    # so only the last U steps of the timed region carry them), and one plain
-    # step for the remainder
-    U = max(1, min(args.unroll, args.steps))
+    # U steps per graph, a whole number of passes over the weight copies
+    U = copies * max(1, math.ceil(min(args.unroll, steps) / copies))
+    K = steps
+    n_u, rem = divmod(K, U)
     probes = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(U)]
-    g_u = torch.cuda.CUDAGraph()
-    g_p = torch.cuda.CUDAGraph()
-    g_1 = torch.cuda.CUDAGraph()
-    main.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(main):
-        with torch.cuda.graph(g_u, stream=main):
-            for _ in range(U):
-                layer.forward(main)
-        with torch.cuda.graph(g_p, stream=main):
-            for i in range(U):
-                layer.forward(main, probes=probes[i])
-        with torch.cuda.graph(g_1, stream=main):
-            layer.forward(main)
+
+    def capture(n, probed=False):
+        g = torch.cuda.CUDAGraph()
+        main.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(main):
+            with torch.cuda.graph(g, stream=main):
+                for i in range(n):
+                    layers[i % copies].forward(main, probes=probes[i] if probed else None)
+        return g
+    g_u = capture(U)
+    g_r = capture(rem) if rem else None
+    g_p = capture(U, probed=True)
     torch.cuda.synchronize()
 
     with torch.cuda.stream(main):
-        for _ in range(args.warmup):
-            g_1.replay()
+        for _ in range(max(1, math.ceil(warmup / U))):
+            g_u.replay()
     torch.cuda.synchronize()
 
-    K = args.steps
-    n_u, rem = divmod(K - U, U) if K >= U else (0, K)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(clocks_local)
     time.sleep(0.3)  # let the sampler start
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.time()
     ev0.record(main)
+    if args.nvtx:
+        torch.cuda.nvtx.range_push("moe_steady_state")
     with torch.cuda.stream(main):
-        for _ in range(rem):
-            g_1.replay()
         for _ in range(n_u):
             g_u.replay()
-        if K >= U:
-            g_p.replay()
+        if g_r is not None:
+            g_r.replay()
+    if args.nvtx:
+        torch.cuda.nvtx.range_pop()
     ev1.record(main)
     torch.cuda.synchronize()
     t1 = time.time()
     barrier(world)
     clk = clocks.stop(t0, t1)
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
     if capi.device_error(main) != 0:
         raise RuntimeError("device error in the timed region")
 
-    # per-kernel durations of the last U launches inside the timed region
+    # kernel durations: the probed graph (the same U steps with events around
+    # the two GEMMs on the main stream), replayed right after the timed region
+    with torch.cuda.stream(main):
+        g_p.replay()
+    torch.cuda.synchronize()
+
     def avg_us(a, b):
-        return 1e3 * sum(p[a].elapsed_time(p[b]) for p in probes) / U if K >= U else float("nan")
+        return 1e3 * sum(p[a].elapsed_time(p[b]) for p in probes) / U
     s1_us, wait_us, s2_us = avg_us(0, 1), avg_us(1, 2), avg_us(2, 3)
     peak, peak_kind = peaks()
     tpeak, tpeak_src = tensor_peak(cfg.dtype)
@@ -353,85 +386,18 @@ def run_ours(args):
     achieved = ab[dom] / (dom_us * 1e-6) / 1e9
     traffic = recorded_traffic(kname, cfg.name)
     step_s = ms / 1e3 / K
-
-    # e2e with host buffers, every step: H2D of the step's inputs from pinned
-    # memory, the step, D2H of its output (StepPipeline below; eager for comparison)
-    # step inputs copied from pinned host memory: the activations the step
-    # reads (bf16 x when the step quantises it, else x in the layer's format),
-    # and the logits unless the step starts from the router linear, which
-    # reads bf16 x (the same tensor for a bf16 layer or with --quantize-x)
-    names = ["x_r" if args.quantize_x else "x"]
-    if not args.quantize_x and inp.get("x_scale") is not None:
-        names.append("x_scale")
-    if args.router_gemm:
-        if cfg.dtype != "bf16" and not args.quantize_x:
-            names.append("x_r")
-    else:
-        names.append("logits")
-    hosts = [inp[n].cpu().pin_memory() for n in names]
-    out_h = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-    E2E = args.e2e_steps
-
-    def e2e_run(step):
-        """E2E steps of: H2D copies of the inputs, one layer step, D2H copy of
-        the output, all on the main stream; device time between two events."""
-        with torch.cuda.stream(main):
-            for _ in range(3):
-                for n, hsrc in zip(names, hosts):
-                    inp[n].copy_(hsrc, non_blocking=True)
-                step()
-                out_h.copy_(layer.out, non_blocking=True)
-        torch.cuda.synchronize()
-        barrier(world)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(main)
-        with torch.cuda.stream(main):
-            for _ in range(E2E):
-                for n, hsrc in zip(names, hosts):
-                    inp[n].copy_(hsrc, non_blocking=True)
-                step()
-                out_h.copy_(layer.out, non_blocking=True)
-        e1.record(main)
-        torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1), world)
-
-    # the serving path (StepPipeline): every step's inputs copied in and its
-    # output copied out, the copies of neighbouring steps overlapping the step
-    pipe = StepPipeline(layer, names, stream=main)
-    outs = [out_h, torch.empty_like(out_h).pin_memory()]
-    pipe.run([hosts] * 3, [outs[i % 2] for i in range(3)])
-    torch.cuda.synchronize()
-    barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e0.record(main)
-    done = pipe.run([hosts] * E2E, [outs[i % 2] for i in range(E2E)])
-    e1 = torch.cuda.Event(enable_timing=True)
-    main.wait_event(done)
-    e1.record(main)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    del pipe
-    eager_ms = e2e_run(lambda: layer.forward(main))  # one step at a time, eager C-ABI calls, serial copies
-    barrier(world)
-
-    result = {
-        "metric": METRIC,
+    layer = layers[0]
+    res = {
         "value": job_tokens_per_s(cfg.T, world, K, ms),
-        "unit": UNIT,
-        "n_gpus": world,
-        "steps": K,
-        "warmup": args.warmup,
         "ms_per_step": ms / K,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        "steps": K,
         "dtype": cfg.dtype,
-        "data": "synthetic",
         "config": {"workload": workload_desc(cfg) + (" +router_gemm" if args.router_gemm else "")
                    + (" +quantize_x" if args.quantize_x else "") + (" +fused_shared" if args.fused_shared else ""),
-                   "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T,
-                   "parallelism": f"replicas{world}", "l2": l2_note(ab["layer"]), "graph": f"CUDA graphs of {U} steps; the last {U} carry timing events",
+                   "global_batch": cfg.T * world, "tokens_per_gpu": cfg.T, "parallelism": f"replicas{world}",
+                   "l2": l2_note(ab["layer"], copies), "weight_copies": copies,
+                   "graph": f"CUDA graphs of {U} steps, no timing events inside the timed region; kernel times from "
+                            f"one probed replay of {U} steps right after it",
                    "block_m": layer.bm, "active_experts": ab["active_experts"]},
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
@@ -444,22 +410,119 @@ def run_ours(args):
                            "binding": "hbm" if ab["layer"] / (peak * 1e9) >= ab["flops"] / (tpeak * 1e12)
                            else "tensor"},
         "kernels_us": {"stage1": s1_us, "addend_wait": wait_us, "stage2": s2_us,
-                       "note": "from the last U steps, whose graph carries timing events"},
-        "e2e": {"value": job_tokens_per_s(cfg.T, world, E2E, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": sum(hs.numel() * hs.element_size() for hs in hosts),
-                "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": E2E,
-                "api": "StepPipeline.run: per step H2D copies (pinned) -> graph of the step -> D2H copy (pinned), "
-                       "the copies of steps i+1 and i-1 overlapping step i on a copy stream",
-                "eager": {"value": job_tokens_per_s(cfg.T, world, E2E, eager_ms),
-                          "api": "layer.forward() per step (eager C-ABI calls), the same copies serialised with it"}},
+                       "note": "one probed replay of the graph after the timed region"},
         "gpu_launches": K * layer.launches_per_step,
         "clocks": clk,
     }
+    del g_u, g_r, g_p
+    if e2e_steps <= 0:
+        return res, inp
+
+    # e2e through the serving loop (StepPipeline): every step copies its inputs
+    # in from pinned host memory and its output back out, the copies of steps
+    # i+1 and i-1 overlapping step i on a copy stream; eager C-ABI calls with
+    # the same copies serialised for comparison
+    names = ["x_r" if args.quantize_x else "x"]
+    if not args.quantize_x and inp.get("x_scale") is not None:
+        names.append("x_scale")
+    if args.router_gemm:
+        if cfg.dtype != "bf16" and not args.quantize_x:
+            names.append("x_r")
+    else:
+        names.append("logits")
+    hosts = [inp[n].cpu().pin_memory() for n in names]
+    out_h = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    pipe = StepPipeline(layer, names, stream=main)
+    outs = [out_h, torch.empty_like(out_h).pin_memory()]
+    pipe.run([hosts] * 3, [outs[i % 2] for i in range(3)])
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    done = pipe.run([hosts] * e2e_steps, [outs[i % 2] for i in range(e2e_steps)])
+    e1 = torch.cuda.Event(enable_timing=True)
+    main.wait_event(done)
+    e1.record(main)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    del pipe
+
+    def eager_step():
+        for n, hsrc in zip(names, hosts):
+            inp[n].copy_(hsrc, non_blocking=True)
+        layer.forward(main)
+        out_h.copy_(layer.out, non_blocking=True)
+    with torch.cuda.stream(main):
+        for _ in range(3):
+            eager_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    with torch.cuda.stream(main):
+        for _ in range(e2e_steps):
+            eager_step()
+    e1.record(main)
+    torch.cuda.synchronize()
+    eager_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    res["e2e"] = {"value": job_tokens_per_s(cfg.T, world, e2e_steps, e2e_ms), "unit": UNIT,
+                  "h2d_bytes_per_step": sum(hs.numel() * hs.element_size() for hs in hosts),
+                  "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps,
+                  "api": "StepPipeline.run: per step H2D copies (pinned) -> graph of the step -> D2H copy (pinned), "
+                         "the copies of steps i+1 and i-1 overlapping step i on a copy stream"
+                         + ("" if copies == 1 else "; one weight copy (the device-timed value cycles "
+                            f"{copies})"),
+                  "eager": {"value": job_tokens_per_s(cfg.T, world, e2e_steps, eager_ms),
+                            "api": "layer.forward() per step (eager C-ABI calls), the same copies serialised "
+                                   "with it"}}
+    return res, inp
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    cfg = configs.CONFIGS[args.config]
+    res, inp = measure(cfg, args, dev, world, args.steps, args.warmup, args.e2e_steps, local)
+    result = {
+        "metric": METRIC,
+        "value": res["value"],
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic",
+    }
+    for k in ("config", "roofline", "layer_roofline", "kernels_us", "e2e", "gpu_launches", "clocks"):
+        if k in res:
+            result[k] = res[k]
+    extra = [w for w in (args.extra.split(",") if args.extra and args.extra != "none" else []) if w != args.config]
+    if extra:
+        result["extra"] = {}
+        for name in extra:
+            ecfg = configs.CONFIGS[name]
+            steps = max(args.steps, args.extra_min_steps)
+            r, _ = measure(ecfg, args, dev, world, steps, args.warmup, 0, local)
+            result["extra"][name] = {k: r[k] for k in ("value", "ms_per_step", "steps", "dtype", "config", "roofline",
+                                                        "layer_roofline", "kernels_us", "gpu_launches", "clocks")}
+            result["gpu_launches"] += r["gpu_launches"]
+        result["gpu_launches_note"] = "headline steps plus the extra workloads' steps"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, inp, min_s=10.0, max_s=30.0)
+        result["cpu_baseline"] = cpu_baseline(cfg, synth.oracle_view(inp), min_s=10.0, max_s=30.0)
     if rank == 0:
         print(json.dumps(result), flush=True)
-    del g_u, g_p, g_1
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -468,89 +531,73 @@ def run_ours(args):
 # ----------------------------------------------------------------- oracle
 
 
-def _oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
 def cpu_baseline(cfg, inp, min_s: float, max_s: float):
-    """The CPU oracle, as it stands, on whole steps of the same workload:
-    repeated over all T tokens until min_s has passed (at most max_s)."""
+    """The C++ oracle, as it stands, on the host threads: whole-token layer
+    forwards (routing, shared expert with its gate, every routed expert, the
+    one bf16 rounding) on a bounded subset of the workload's tokens, grown
+    until min_s has passed (at most about max_s)."""
     import oracle
-    ov = synth.oracle_view(inp)
     c = cfg.as_dict()
-    tokens = 0
+    threads = oracle.num_threads()
+    rng = np.random.default_rng(0)
+    order = rng.permutation(cfg.T)
+    done = 0
+    n = threads
     t0 = time.time()
     while True:
-        oracle.moe_layer(c, ov)
-        tokens += cfg.T
+        toks = order[done % cfg.T: done % cfg.T + n]
+        oracle.moe_layer(c, inp, tokens=toks, threads=threads)
+        done += len(toks)
         el = time.time() - t0
-        if el >= min_s or el + el / max(tokens // cfg.T, 1) > max_s:
+        per = el / done
+        if el >= min_s or el + per * n > max_s:
             break
-    return {"value": tokens / el, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{tokens // cfg.T} full step(s) of {cfg.T} tokens, {el:.1f} s (numpy float64; BLAS "
-                      f"matrix-vector products threaded, the rest single-threaded)"}
+        n = max(threads, min(4 * threads, int((min_s - el) / per) // threads * threads))
+    return {"value": done / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} of the workload's {cfg.T} tokens (seeded random subset), each a whole-layer forward "
+                      f"through the plain C++ oracle (float64, OpenMP over tokens, {threads} threads), {el:.1f} s"}
 
 
 def run_reference(args):
+    """The oracle as the reference arm: each step is one batch of expert calls
+    (one unit per host thread: a routed expert of one (token, slot) pair, or
+    one token's shared expert; top_k + 1 units make one token), cycling
+    through the workload's tokens."""
     world, rank, _ = dist_env()
     if rank != 0:
         return
     import oracle
+    from oracle import cpp
     cfg = configs.CONFIGS[args.config]
     inp = synth.oracle_view(synth.make_layer_inputs(cfg))
-    c = cfg.as_dict()
-    # one unit = one expert MLP of one (token, slot) pair, or one token's shared
-    # expert; a token is top_k + 1 units. Steps cycle through the workload.
-    cb = inp.get("correction_bias")
-    ids, w = oracle.route(c, inp["logits"].numpy(), None if cb is None else cb.numpy())
-    mx = cfg.dtype in ("mxfp8", "mxfp4")
-    afmt = "mxfp8" if mx else cfg.dtype  # activations and h (MXFP4 layers: MXFP8)
-    x = oracle.decode_operand(inp["x"], afmt, inp["x_scale"] if mx else None)
-    s_x = inp["x_scale"].reshape(-1).double().numpy() if cfg.dtype == "fp8" else None
+    threads = oracle.num_threads()
+    lu = cpp.LayerUnits(cfg.as_dict(), inp, threads=threads)
     units = [(t, j) for t in range(cfg.T) for j in range(-1, cfg.top_k)]
+    pos = 0
 
-    def wts(name, e=None):
-        """Decoded weights and the fp8 per-matrix scale (1 otherwise)."""
-        t, sc = inp[name], inp.get(name + "_scale")
-        if e is not None:
-            t = t[e]
-        if mx:
-            return oracle.decode_operand(t, cfg.dtype, sc if e is None else sc[e]), 1.0
-        if cfg.dtype == "fp8":
-            return oracle.decode_operand(t, "fp8"), float(sc.reshape(-1)[0 if e is None else e])
-        return oracle.decode_operand(t, cfg.dtype), 1.0
+    def step():
+        nonlocal pos
+        batch = [units[(pos + i) % len(units)] for i in range(threads)]
+        pos += threads
+        lu.run(batch)
 
-    def step(i):
-        t, j = units[i % len(units)]
-        sx = 1.0 if s_x is None else float(s_x[t])
-        if j < 0:
-            (w13, s13), (w2, s2), inter = wts("w13s"), wts("w2s"), cfg.Is
-        else:
-            e = ids[t, j]
-            (w13, s13), (w2, s2), inter = wts("w13", e), wts("w2", e), cfg.I
-        oracle.expert_forward(x[t], w13, w2, inter, afmt, sx, s13, s2)
-
-    for i in range(args.warmup):
-        step(i)
+    for _ in range(args.warmup):
+        step()
     t0 = time.time()
-    for i in range(args.steps):
-        step(args.warmup + i)
+    for _ in range(args.steps):
+        step()
     el = time.time() - t0
-    tok = args.steps / (cfg.top_k + 1)
+    tok = args.steps * threads / (cfg.top_k + 1)
     val = tok / el
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.T, "parallelism": "cpu"},
-        "cpu_baseline": {"value": val, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-                         "sample": f"each step = one expert MLP of one (token, slot) pair or one shared expert "
-                                   f"({cfg.top_k + 1} units = 1 token); {args.steps} units"},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"each step = {threads} expert calls in parallel through the plain C++ oracle "
+                                   f"(a routed expert of one (token, slot) pair or one token's shared expert; "
+                                   f"{cfg.top_k + 1} calls = 1 token); {args.steps} steps"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

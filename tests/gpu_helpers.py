@@ -182,7 +182,8 @@ def gpu_h_values(layer, rows, shared=False):
     vals = _e4m3_values(codes)
     sc = layer.h_scale_s if shared else layer.h_scale
     if cfg.dtype == "fp8":
-        return vals * sc.cpu().numpy()[rows].astype(np.float64)[:, None]
+        # the e4m3 values of the codes (the GPU's row scale, continuous, is returned apart)
+        return vals, sc.cpu().numpy()[rows].astype(np.float64)
     ncol = codes.shape[1]
     bm = layer.bm
     rr = np.asarray(rows) % bm
@@ -207,8 +208,19 @@ def _tie_distance(a):
 def h_flip_check(cfg, h_gpu, h_raw, h_q):
     """Codes of the GPU's h [..., n] that differ from the oracle's h_q, each
     checked to be the other rounding of a tie of the oracle's unquantised
-    h_raw; returns |h_gpu - h_q| (zero where they agree)."""
-    d = h_gpu - h_q
+    h_raw; returns the value difference those codes make, |dh| (zero where the
+    codes agree). fp8: h_gpu is (e4m3 values of the codes, the GPU's row
+    scales); the per-row scale amax/448 is continuous and may differ from the
+    oracle's in its last bit, which scales a whole row by about 1e-7 (inside
+    the output tolerance), so codes are compared, and a differing code counts
+    at the oracle's scale."""
+    if cfg.dtype == "fp8":
+        q_gpu, _ = h_gpu
+        amax = np.max(np.abs(h_raw), axis=-1, keepdims=True)
+        s_or = np.where(amax > 0, oracle.fp32_round(amax / 448.0), 1.0)
+        d = (q_gpu.reshape(h_q.shape) - h_q / s_or) * s_or
+    else:
+        d = h_gpu - h_q
     flips = d != 0
     if not flips.any():
         return np.zeros_like(d)
@@ -258,7 +270,8 @@ def quantised_layer_allowance(cfg, layer, inp, tokens, ref):
     slots = (np.asarray(tokens)[:, None] * k + np.arange(k)[None, :]).reshape(-1)
     rows = row_of[slots]
     assert np.all(rows >= 0)
-    hg = gpu_h_values(layer, rows).reshape(len(tokens), k, I)
+    hg = gpu_h_values(layer, rows)
+    hg = (hg[0].reshape(len(tokens), k, I), hg[1]) if cfg.dtype == "fp8" else hg.reshape(len(tokens), k, I)
     d_r = h_flip_check(cfg, hg, ref["h_raw"], ref["h_q"])
     hs = gpu_h_values(layer, np.asarray(tokens), shared=True)
     d_s = h_flip_check(cfg, hs, ref["h_raw_shared"], ref["h_q_shared"])

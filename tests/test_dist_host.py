@@ -110,9 +110,14 @@ def test_mx_and_fp8_bytes_count_their_scales():
     assert synth.activation_bytes("mxfp4", 10, 4096) == 10 * 4096 + 10 * 128
 
 
-def test_l2_note_is_true_to_the_step_size():
+def test_weight_copies_put_every_step_over_three_l2s():
+    """Steps that read less than 3x the 126 MB L2 cycle through enough weight
+    copies that every step's weights come from HBM; larger steps use one."""
     sys.path.insert(0, ROOT)
     import bench
-    assert "come from HBM" in bench.l2_note(0.81e9)
-    assert "may still be in L2" in bench.l2_note(200e6)
-    assert "L2-resident" in bench.l2_note(1.8e6)
+    for step in (1.8e6, 138e6, 230e6, 0.81e9, 11.6e9):
+        n = bench.weight_copies(step)
+        assert n * step >= 3 * bench.L2_BYTES
+        assert n == 1 or (n - 1) * step < 3 * bench.L2_BYTES
+        assert "come from HBM" in bench.l2_note(step, n)
+    assert bench.weight_copies(0.81e9) == 1 and bench.weight_copies(1.8e6) == 210

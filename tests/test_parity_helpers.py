@@ -39,9 +39,15 @@ def test_a_code_taken_at_a_tie_is_accepted_and_measured(fmt):
     h_gpu = h_q.copy()
     sc = s[1, 0] if fmt == "fp8" else s[1, 5]
     h_gpu[1, 5] = _other_rounding(np.array([h_raw[1, 5] / sc]))[0] * sc
-    d = h_flip_check(cfg, h_gpu, h_raw, h_q)
-    assert np.count_nonzero(d) == 1 and d[1, 5] == pytest.approx(step * sc)
-    assert np.all(h_flip_check(cfg, h_q, h_raw, h_q) == 0)
+    if fmt == "fp8":  # codes (e4m3 values) and the GPU's row scales, one ulp off the oracle's
+        gs = s[:, 0] * (1 + 2.0 ** -23)
+        d = h_flip_check(cfg, (h_gpu / s, gs), h_raw, h_q)
+        d0 = h_flip_check(cfg, (h_q / s, gs), h_raw, h_q)
+    else:
+        d = h_flip_check(cfg, h_gpu, h_raw, h_q)
+        d0 = h_flip_check(cfg, h_q, h_raw, h_q)
+    assert np.count_nonzero(d) == 1 and abs(d[1, 5]) == pytest.approx(step * sc)
+    assert np.all(d0 == 0)
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "mxfp8"])
@@ -54,5 +60,8 @@ def test_a_code_differing_away_from_a_tie_is_rejected(fmt):
     i = np.unravel_index(np.argmin(np.abs(h_raw - h_q) / np.maximum(np.abs(h_raw), 1e-9)), h_raw.shape)
     h_gpu = h_q.copy()
     h_gpu[i] = h_q[i] * (1 + 2.0 ** -3)
+    if fmt == "fp8":
+        s = oracle.fp32_round(np.max(np.abs(h_raw), axis=-1, keepdims=True) / 448.0)
+        h_gpu = (h_gpu / s, s[:, 0])
     with pytest.raises(AssertionError):
         h_flip_check(cfg, h_gpu, h_raw, h_q)
