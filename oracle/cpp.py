@@ -86,6 +86,7 @@ def lib():
             "orc_shared_gate": (None, [P, P, i32, i32, i32, i32, P]),
             "orc_expert_forward": (None, [P, P, P, i32, i32, i32, f64, f64, f64, P, P]),
             "orc_moe_layer": (i32, [ctypes.POINTER(OrcLayer), P, i32, i32, i32, P, P, P, P, P, P]),
+            "orc_moe_layer_h": (i32, [ctypes.POINTER(OrcLayer), P, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]),
             "orc_layer_units": (i32, [ctypes.POINTER(OrcLayer), P, P, P, i32, i32, P]),
             "orc_num_threads": (i32, []),
         }
@@ -470,11 +471,14 @@ def _layer_struct(cfg: dict, inp: dict):
     return L, keep
 
 
-def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False, threads: int = 0) -> dict:
+def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False, threads: int = 0,
+              want_h: bool = False) -> dict:
     """The layer, token by token (see orc_moe_layer in moe_oracle.cpp).
     Same keys in and out as the numpy oracle's ``moe_layer``; ``threads`` = 0
-    uses every host thread."""
-    T, H, k = cfg["T"], cfg["H"], cfg["top_k"]
+    uses every host thread. ``want_h`` adds the stage-1 values of the
+    computed tokens: ``h_raw`` / ``h_q`` [n, k, I] per routed slot (before and
+    after quantisation) and ``h_raw_shared`` / ``h_q_shared`` [n, Is]."""
+    T, H, k, I, Is = cfg["T"], cfg["H"], cfg["top_k"], cfg["I"], cfg["Is"]
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     tok = np.ascontiguousarray(tokens.astype(np.int32))
     L, _keep = _layer_struct(cfg, inp)
@@ -485,11 +489,15 @@ def moe_layer(cfg: dict, inp: dict, tokens=None, shared_fused: bool = False, thr
     addend = np.empty((n, H), np.float64)
     routed = np.empty((n, H), np.float64)
     out = np.empty((n, H), np.float64)
-    r = lib().orc_moe_layer(ctypes.byref(L), _ptr(tok), n, int(shared_fused), int(threads), _ptr(ids), _ptr(w),
-                            _ptr(g), _ptr(addend), _ptr(routed), _ptr(out))
+    hs = [np.zeros((n, k, I)), np.zeros((n, k, I)), np.zeros((n, Is)), np.zeros((n, Is))] if want_h else [None] * 4
+    r = lib().orc_moe_layer_h(ctypes.byref(L), _ptr(tok), n, int(shared_fused), int(threads), _ptr(ids), _ptr(w),
+                              _ptr(g), _ptr(addend), _ptr(routed), _ptr(out), *[_ptr(a) for a in hs])
     assert r == 0, "invalid layer arguments"
-    return {"topk_ids": ids, "topk_weights": w, "gate": g, "addend": addend, "routed": routed, "out": out,
-            "tokens": tokens}
+    res = {"topk_ids": ids, "topk_weights": w, "gate": g, "addend": addend, "routed": routed, "out": out,
+           "tokens": tokens}
+    if want_h:
+        res.update(h_raw=hs[0], h_q=hs[1], h_raw_shared=hs[2], h_q_shared=hs[3])
+    return res
 
 
 class LayerUnits:

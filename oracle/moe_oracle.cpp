@@ -258,11 +258,15 @@ void expert_hidden(const double* x, const Mat& w13, int I, double s_x, double s_
 // h quantised (quantize_h); y = (W2 . h) * s_w2 (a per-row scale of h is
 // already inside the dequantised h; MX block scales are inside the decoded
 // operands).
+// h_raw / h_q (optional, I values each): the stage-1 value before and after
+// its quantisation.
 void expert_forward(const double* x, const Mat& w13, const Mat& w2, int I, int hmode, double s_x, double s_w13,
-                    double s_w2, double* y) {
+                    double s_w2, double* y, double* h_raw = nullptr, double* h_q = nullptr) {
   std::vector<double> h(I), row(std::max(w13.cols, w2.cols));
   expert_hidden(x, w13, I, s_x, s_w13, h.data(), row.data());
+  if (h_raw) std::memcpy(h_raw, h.data(), sizeof(double) * I);
   quantize_h(h.data(), I, hmode);
+  if (h_q) std::memcpy(h_q, h.data(), sizeof(double) * I);
   for (int n = 0; n < w2.rows; ++n) {
     decode_row(w2, n, row.data());
     y[n] = dot(row.data(), h.data(), I) * s_w2;
@@ -652,8 +656,23 @@ struct OrcLayer {
 // Tokens run in parallel (OpenMP, `threads` threads; 0 = the default); each
 // token's arithmetic is the same whatever the thread count.
 // Returns 0, or -1 for an invalid argument.
+// orc_moe_layer with optional outputs of the stage-1 values: h_raw_r / h_q_r
+// [n_tok, k, I] (each routed slot's h before and after its quantisation) and
+// h_raw_s / h_q_s [n_tok, Is] (the shared expert's; not filled in fused
+// mode). Any of them may be NULL.
+int orc_moe_layer_h(const OrcLayer* L, const int32_t* tokens, int n_tok, int shared_fused, int threads, int32_t* ids,
+                    double* wts, double* gate, double* addend, double* routed, double* out, double* h_raw_r,
+                    double* h_q_r, double* h_raw_s, double* h_q_s);
+
 int orc_moe_layer(const OrcLayer* L, const int32_t* tokens, int n_tok, int shared_fused, int threads, int32_t* ids,
                   double* wts, double* gate, double* addend, double* routed, double* out) {
+  return orc_moe_layer_h(L, tokens, n_tok, shared_fused, threads, ids, wts, gate, addend, routed, out, nullptr,
+                         nullptr, nullptr, nullptr);
+}
+
+int orc_moe_layer_h(const OrcLayer* L, const int32_t* tokens, int n_tok, int shared_fused, int threads, int32_t* ids,
+                    double* wts, double* gate, double* addend, double* routed, double* out, double* h_raw_r,
+                    double* h_q_r, double* h_raw_s, double* h_q_s) {
   const int T = L->T, H = L->H, E = L->E, k = L->top_k, I = L->I, Is = L->Is;
   if (T < 1 || H < 1 || E < 1 || k < 1 || k > E || I < 1 || Is < 1 || L->fmt < 0 || L->fmt > 3) return -1;
   const int fmt = L->fmt;
@@ -738,7 +757,9 @@ int orc_moe_layer(const OrcLayer* L, const int32_t* tokens, int n_tok, int share
         for (int n = 0; n < H; ++n) add[n] += g * (dot(P2 + static_cast<size_t>(n) * I, hh.data(), I) * s2s);
       }
     } else {
-      expert_forward(x.data(), w13s, w2s, Is, hmode, s_x, s13s, s2s, y.data());
+      expert_forward(x.data(), w13s, w2s, Is, hmode, s_x, s13s, s2s, y.data(),
+                     h_raw_s ? h_raw_s + static_cast<size_t>(i) * Is : nullptr,
+                     h_q_s ? h_q_s + static_cast<size_t>(i) * Is : nullptr);
       for (int n = 0; n < H; ++n) add[n] = round_to(g * y[n], kBF16);
     }
 
@@ -747,8 +768,9 @@ int orc_moe_layer(const OrcLayer* L, const int32_t* tokens, int n_tok, int share
       const int e = ids[static_cast<size_t>(t) * k + j];
       const Mat w13 = slice(fmt, L->w13, L->w13_scale, 2 * I, H, e);
       const Mat w2 = slice(fmt, L->w2, L->w2_scale, H, I, e);
+      const size_t hoff = (static_cast<size_t>(i) * k + j) * I;
       expert_forward(x.data(), w13, w2, I, hmode, s_x, scale_of(L->w13_scale, e), scale_of(L->w2_scale, e),
-                     y.data());
+                     y.data(), h_raw_r ? h_raw_r + hoff : nullptr, h_q_r ? h_q_r + hoff : nullptr);
       const double wj = wts[static_cast<size_t>(t) * k + j];
       for (int n = 0; n < H; ++n) acc[n] += wj * y[n];
     }

@@ -560,8 +560,8 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
             if (ncols == BN) tma_load_2d_pair(b_dst, &tmB, fb, kb * KE, row0, pol_x);
             if (MX) {
               const int wt = (expert * g.n_mt + mt) * g.num_kb + kb;
-              tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, wt * 32, pol_w);
-              tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 32, pol_x);
+              tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, wt * 4, pol_w);
+              tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 4, pol_x);
             }
             pending |= 1u << stage;
             pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);

@@ -97,12 +97,13 @@ moe_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const vo
   return MOE_OK;
 }
 
-// Map of an MX scale-tile array (512-byte tiles) as rows of 16 bytes: one
-// 16 x 32 box is one tile, landing dense in shared memory (no swizzle).
+// Map of an MX scale-tile array (512-byte tiles) as rows of 128 bytes: one
+// 128 x 4 box is one tile (four row requests), landing dense in shared memory
+// (no swizzle).
 moe_status_t make_sf_tile_map(CUtensorMap* m, const void* base, size_t tiles) {
-  const cuuint64_t dims[2] = {16, static_cast<cuuint64_t>(tiles) * 32};
-  const cuuint64_t st[1] = {16};
-  const cuuint32_t box[2] = {16, 32};
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(tiles) * 4};
+  const cuuint64_t st[1] = {128};
+  const cuuint32_t box[2] = {128, 4};
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
