@@ -57,12 +57,20 @@ __host__ __device__ constexpr bool is_mx(int kind) { return kind == kMx8 || kind
 // one group from 64 tokens on (registers for the held h values); block-scaled
 // stage 2 at 128 tokens shares three accumulators between its two groups, the
 // scale ring taking TMEM's last columns.
+//
+// Copy issue: a thread needs about 130 cycles to issue one TMA copy, so at
+// 64-token tiles and more, where a stage holds a large token tile too, two
+// producer warps share it: warp 0 loads the weight tile (and its MX scale
+// tile), warp 2 the token tile (and its scale tile); both arm the stage's
+// `full` barrier with their own bytes. Smaller tiles keep one producer warp.
 template <int BN, int KIND, bool S1>
 struct EpiCfg {
   static constexpr bool kMxWide = is_mx(KIND) && BN == 128 && !S1;
   static constexpr int kGroups = (is_mx(KIND) ? (BN <= 32 || !S1) : BN <= 128) ? 2 : 1;
   static constexpr int kAcc = kMxWide ? 3 : 2 * kGroups;
-  static constexpr int kThreads = 64 + kEpiThreads * kGroups;
+  static constexpr bool kSplit = BN >= 64;              // two producer warps
+  static constexpr int kLead = kSplit ? 96 : 64;         // threads before the epilogue warps
+  static constexpr int kThreads = kLead + kEpiThreads * kGroups;
 };
 
 struct GemmArgs {
@@ -184,6 +192,18 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   const int x = e - 1 - 8;
   return x < -127 ? -127 : (x > 127 ? 127 : x);
 }
+
+// mx_exponent from the bits of a finite non-negative amax: the biased
+// exponent field e gives floor(log2 amax) = e - 127 for a normal amax; zero
+// and subnormal amax (e = 0) give -135, clamped to -127 like the definition.
+// (A finite fp32 amax gives at most 254 - 135 = 119.)
+__device__ __forceinline__ int mx_exponent_bits(float amax) {
+  const int x = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
+  return x < -127 ? -127 : (x > 127 ? 127 : x);
+}
+
+// 2^-X as an fp32 number, for X in [-127, 126] (biased exponent 127 - X in [1, 254]).
+__device__ __forceinline__ float pow2_neg(int X) { return __uint_as_float(static_cast<uint32_t>(127 - X) << 23); }
 
 // Quantise the rows of token block `blk` that hold a slot from the
 // unquantised fp32 h to e4m3 with one fp32 scale per row, s = amax / 448
@@ -451,6 +471,8 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
   constexpr int KE = KIND == kBf16 ? 64 : 128;  // K elements per stage
   constexpr int kUmmaKBytes = 32;               // K bytes per MMA: 16 bf16 or 32 e4m3
   constexpr int kMmaM = PAIR ? 2 * kTileM : kTileM;
+  constexpr bool SPLIT = EpiCfg<BN, KIND, S1>::kSplit;
+  constexpr int kLead = EpiCfg<BN, KIND, S1>::kLead;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
   static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
@@ -476,7 +498,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], SPLIT ? 2 : 1);  // each producer warp arms it with its own bytes
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < NACC; ++a) {
@@ -523,8 +545,10 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
   const int total = n_blocks * n_wt;
   const int slots = g.T * g.top_k;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || (SPLIT && warp == 2)) {
+    // ------------------------------------------------------------ producer(s)
+    const bool do_w = !SPLIT || warp == 0;  // weight tile (+ its MX scale tile)
+    const bool do_t = !SPLIT || warp == 2;  // token tile (+ its MX scale tile)
     const uint64_t pol_w = policy_evict_first();  // weights stream through once
     const uint64_t pol_x = policy_evict_last();   // token rows are re-read per weight tile
     int stage = 0;
@@ -534,41 +558,48 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     for (int tile = unit0; tile < total && ok; tile += n_units) {
       const int blk = tile / n_wt;
       const int mt = PAIR ? 2 * (tile - blk * n_wt) + static_cast<int>(rank) : tile - blk * n_wt;
-      const int expert = block_expert_of(g, blk);
+      const int expert = do_w ? block_expert_of(g, blk) : 0;
       const int ncols = block_cols<BN>(g, blk, lane);  // token rows this tile loads and multiplies
       const int my_rows = PAIR ? ncols / 2 : ncols;    // token rows this CTA loads
       const int row0 = blk * BN + (PAIR ? static_cast<int>(rank) * my_rows : 0);
+      // transaction bytes count what this warp's copies read from global
+      // memory: half the shared-memory footprint for the packed e2m1 weight tile
+      uint32_t bytes = 0;
+      if (do_w) bytes += (KIND == kMx4 ? L::kABytes / 2 : L::kABytes) + (MX ? kSfTile : 0);
+      if (do_t) bytes += static_cast<uint32_t>(my_rows) * kTileKBytes + (MX ? kSfTile : 0);
+      // A tile whose token rows come in one box needs lane 0 only: it runs the
+      // tile's stages alone, and the warp re-joins at the tile's end. Short
+      // tiles spread their row boxes over the lanes, stage by stage.
+      const bool solo = ncols == BN || !do_t;
       for (int kb = 0; kb < g.num_kb; ++kb) {
+        if (solo && lane != 0) break;
         uint8_t* a_dst = smem + stage * L::kStageBytes;
         uint8_t* b_dst = a_dst + L::kABytes;
         uint8_t* sfa_dst = b_dst + L::kBBytes;
         uint8_t* sfb_dst = sfa_dst + kSfTile;
         if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!solo) ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        // transaction bytes count what the copies read from global memory:
-        // half the shared-memory footprint for the packed e2m1 weight tile
-        uint32_t bytes = (KIND == kMx4 ? L::kABytes / 2 : L::kABytes) + static_cast<uint32_t>(my_rows) * kTileKBytes;
-        if (MX) bytes += 2 * kSfTile;
         if constexpr (PAIR) {
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
           if (lane == 0) {
             pending &= ~(1u << stage);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);  // both CTAs' copies
-            if (S1) tma_load_5d_pair(a_dst, &tmA, fb, kb * KE, 0, 0, mt * 4, expert, pol_w);
-            else tma_load_3d_pair(a_dst, &tmA, fb, kb * KE, mt * kTileM, expert, pol_w);
-            if (ncols == BN) tma_load_2d_pair(b_dst, &tmB, fb, kb * KE, row0, pol_x);
-            if (MX) {
-              const int wt = (expert * g.n_mt + mt) * g.num_kb + kb;
-              tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, wt * 4, pol_w);
-              tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 4, pol_x);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);  // both CTAs' copies of this kind
+            if (do_w) {
+              if (S1) tma_load_5d_pair(a_dst, &tmA, fb, kb * KE, 0, 0, mt * 4, expert, pol_w);
+              else tma_load_3d_pair(a_dst, &tmA, fb, kb * KE, mt * kTileM, expert, pol_w);
+              if (MX) tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, ((expert * g.n_mt + mt) * g.num_kb + kb) * 4, pol_w);
+            }
+            if (do_t) {
+              if (ncols == BN) tma_load_2d_pair(b_dst, &tmB, fb, kb * KE, row0, pol_x);
+              if (MX) tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 4, pol_x);
             }
             pending |= 1u << stage;
             pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           }
-          __syncwarp();
+          if (!solo) __syncwarp();
           // a short tile: this CTA's token rows in 8-row boxes, issued by the lanes
-          if (ncols < BN) {
+          if (do_t && ncols < BN) {
             for (int q = lane; q < my_rows / 8; q += 32)
               tma_load_2d_pair(b_dst + q * 8 * kTileKBytes, &tmB16, fb, kb * KE, row0 + q * 8, pol_x);
           }
@@ -576,23 +607,28 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           if (lane == 0) {
             pending &= ~(1u << stage);
             mbar_arrive_expect_tx(&full[stage], bytes);
-            if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
-            else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
-            // token rows as one box when the tile is full (B from x, the sorted copy, or h)
-            if (ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
-            if (MX) {
-              const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
-              bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
-              bulk_load(sfb_dst, (S1 ? g.xsf : g.hsf) + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile,
-                        kSfTile, &full[stage], pol_x);
+            if (do_w) {
+              if (S1) tma_load_5d(a_dst, &tmA, &full[stage], kb * KE, 0, 0, mt * 4, expert, pol_w);
+              else tma_load_3d(a_dst, &tmA, &full[stage], kb * KE, mt * kTileM, expert, pol_w);
+              if (MX) {
+                const size_t wt = (static_cast<size_t>(expert) * g.n_mt + mt) * g.num_kb + kb;
+                bulk_load(sfa_dst, g.wsf + wt * kSfTile, kSfTile, &full[stage], pol_w);
+              }
+            }
+            if (do_t) {
+              // token rows as one box when the tile is full (B from x, the sorted copy, or h)
+              if (ncols == BN) tma_load_2d(b_dst, &tmB, &full[stage], kb * KE, blk * BN, pol_x);
+              if (MX)
+                bulk_load(sfb_dst, (S1 ? g.xsf : g.hsf) + (static_cast<size_t>(blk) * g.num_kb + kb) * kSfTile,
+                          kSfTile, &full[stage], pol_x);
             }
             pending |= 1u << stage;
             pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           }
-          __syncwarp();
+          if (!solo) __syncwarp();
           // a short tile: its token rows in 16-row boxes, issued by the lanes of
           // the warp (the barrier was armed above with the stage's full byte count)
-          if (ncols < BN) {
+          if (do_t && ncols < BN) {
             for (int q = lane; q < ncols / 16; q += 32)
               tma_load_2d(b_dst + q * 16 * kTileKBytes, &tmB16, &full[stage], kb * KE, blk * BN + q * 16, pol_x);
           }
@@ -601,6 +637,11 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           stage = 0;
           phase ^= 1u;
         }
+      }
+      if (solo) {  // the other lanes take lane 0's ring position and status
+        stage = __shfl_sync(0xffffffffu, stage, 0);
+        phase = __shfl_sync(0xffffffffu, phase, 0);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
       __syncwarp();
     }
@@ -617,7 +658,10 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // (a pair's MMAs are all issued by rank 0)
+    // (a pair's MMAs are all issued by rank 0). The warp computes each tile's
+    // token-column count together; lane 0 alone then runs the tile's K stages
+    // (issue is one thread's work, and per-stage warp shuffles and syncs cost
+    // as much as an MMA issue).
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -625,21 +669,18 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
     int j = 0;  // local tile counter: accumulator j % NACC, use (j / NACC)
     const bool issuer = !PAIR || rank == 0;
     for (int tile = unit0; issuer && tile < total; tile += n_units, ++j) {
-      const int acc = j % NACC;
-      const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
       const int ncols = block_cols<BN>(g, tile / n_wt, lane);
-      const uint32_t idesc = FP8 ? idesc_e4m3(kMmaM, ncols) : idesc_bf16(kMmaM, ncols);
-      if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < g.num_kb; ++kb) {
-        if (lane == 0) ok = mbar_wait(&full[stage], phase, abort_flag);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
+      if (lane == 0) {
+        const int acc = j % NACC;
+        const uint32_t acc_phase = static_cast<uint32_t>(j / NACC) & 1u;
+        const uint32_t idesc = FP8 ? idesc_e4m3(kMmaM, ncols) : idesc_bf16(kMmaM, ncols);
+        ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        if (ok) tc_fence_after();
+        for (int kb = 0; ok && kb < g.num_kb; ++kb) {
+          ok = mbar_wait(&full[stage], phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
           const uint64_t adesc = sw128_kmajor_desc(a_addr);
           const uint64_t bdesc = sw128_kmajor_desc(a_addr + L::kABytes);
@@ -684,34 +725,33 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           } else {
             umma_commit(&empty[stage]);
           }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+        if (ok) {
+          if constexpr (PAIR) {
+            umma_commit_pair(acc_full_r[0] + 8u * static_cast<uint32_t>(acc));
+            umma_commit_pair(acc_full_r[1] + 8u * static_cast<uint32_t>(acc));
+          } else {
+            umma_commit(&acc_full[acc]);
+          }
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      if (lane == 0) {
-        if constexpr (PAIR) {
-          umma_commit_pair(acc_full_r[0] + 8u * static_cast<uint32_t>(acc));
-          umma_commit_pair(acc_full_r[1] + 8u * static_cast<uint32_t>(acc));
-        } else {
-          umma_commit(&acc_full[acc]);
-        }
-      }
-      __syncwarp();
     }
     if (!ok && lane == 0) {
       if constexpr (PAIR) umma_commit_pair(mapa_shared(smem_u32(drain), 0));
       else umma_commit(drain);
       drain_wait(drain, 0);
     }
-  } else {
+  } else if (warp >= kLead / 32) {
     // ------------------------------------------------------------ epilogue
-    const int grp = (warp - 2) >> 2;              // epilogue group: tiles j with j % G == grp
+    const int grp = (warp - kLead / 32) >> 2;     // epilogue group: tiles j with j % G == grp
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
-    const int et = threadIdx.x - 64 - kEpiThreads * grp;  // 0..127 inside the group
+    const int et = threadIdx.x - kLead - kEpiThreads * grp;  // 0..127 inside the group
     const int bar_id = 1 + grp;                   // named barrier of this group
     int* gsm = group_base + grp * L::kGroupWords;
     volatile int* ok_sm = gsm;
@@ -793,7 +833,11 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
               gt *= sc;
               up *= sc;
             }
-            const float hv = gt / (1.0f + expf(-gt)) * up;
+            // MXFP8 h is quantised to three mantissa bits next: the fast
+            // exponential and division (relative error ~1e-6, as small as the
+            // fp32 accumulation's) keep this loop short; bf16 and fp8 h use
+            // the exact ones
+            const float hv = MX ? __fdividef(gt, 1.0f + __expf(-gt)) * up : gt / (1.0f + expf(-gt)) * up;
             if (!MX && feat < g.I) {
               if (FP8) g.h32[static_cast<size_t>(r) * g.I + feat] = hv;
               else g.h[static_cast<size_t>(r) * g.I + feat] = __float2bfloat16_rn(hv);
@@ -824,8 +868,8 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
             if (2 * i >= ncols) continue;
             const int c = 2 * i + (lo ? 0 : 1);
             const float amax = fmaxf(amax_part[q * BN + c], amax_part[(q ^ 1) * BN + c]);
-            const int X = mx_exponent(amax);
-            const float v = ldexpf(hv_keep[i], -X);
+            const int X = mx_exponent_bits(amax);
+            const float v = hv_keep[i] * pow2_neg(X);  // exact: a power of two in the normal range
             const uint8_t code = static_cast<uint8_t>(cvt_e4m3x2(v, 0.f) & 0xFF);
             if (feat < g.I) g.hq[static_cast<size_t>(blk * BN + c) * g.I + feat] = code;
             if ((q & 1) == 0 && (lane & 15) == 0)

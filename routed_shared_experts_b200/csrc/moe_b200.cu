@@ -129,18 +129,19 @@ constexpr int pair_stages() {
     return ST;
 }
 
-// Whether a GEMM runs on CTA pairs (one MMA of M = 256 per pair, each SM
-// loading its 128 weight rows and half the token tile): 128-token tiles, an
-// even number of 128-row weight sub-tiles, not the fp8 stage 1 (its per-row
-// quantisation of h follows a grid barrier in a cooperative launch). At
-// 128-token tiles the kernels are paced by the operand bytes each SM brings
-// into shared memory, and a pair brings 24 KB + scales per stage for what one
-// CTA needed 32 KB. MOE_B200_PAIR=0 in the environment selects single CTAs
-// everywhere (same results).
+// Whether a GEMM runs on CTA pairs (one MMA of M = 256 per 2-CTA cluster,
+// each SM loading its 128 weight rows and half the token tile): opt-in with
+// MOE_B200_PAIR=1, for 128-token tiles whose weight rows split into an even
+// number of 128-row tiles, never the fp8 stage 1 (its per-row quantisation of
+// h follows a grid barrier in a cooperative launch). Measured on the prefill
+// layers, the pairs run a few percent slower than one CTA per tile: each
+// stage costs about the same number of issued copies per SM either way, and
+// the issue of copies and MMAs, not the operand bytes, paces these kernels.
+// Results do not depend on the choice.
 bool use_pair(int dtype, int bm, int n_mt, bool s1) {
   static const bool enabled = [] {
     const char* v = getenv("MOE_B200_PAIR");
-    return !(v && v[0] == '0');
+    return v && v[0] == '1';
   }();
   return enabled && bm == 128 && n_mt % 2 == 0 && !(s1 && dtype == MOE_DT_FP8_E4M3);
 }
