@@ -10,6 +10,7 @@
 namespace moe {
 
 constexpr int kSortThreads = 1024;
+constexpr int kSortBatch = 8;  // 32-slot steps whose ids a warp loads at once
 
 struct SortArgs {
   const int32_t* ids;  // [N] flat slots f = t*k + j
@@ -53,17 +54,27 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
   __syncthreads();
 
-  // 1. per-warp counts
-  for (int b = f0; b < f1; b += 32) {
-    const int f = b + lane;
-    int e = f < f1 ? a.ids[f] : -1;
-    if (e >= E || (f < f1 && e < 0)) {
-      set_device_error(kErrExpertRange);
-      e = -1;
+  // 1. per-warp counts; the ids of kSortBatch steps are loaded before any is
+  // used, so that a warp keeps that many loads in flight
+  for (int b0 = f0; b0 < f1; b0 += 32 * kSortBatch) {
+    int ev[kSortBatch];
+#pragma unroll
+    for (int u = 0; u < kSortBatch; ++u) {
+      const int f = b0 + 32 * u + lane;
+      ev[u] = f < f1 ? a.ids[f] : -1;
     }
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0) my_cnt_row[e] += __popc(peers);
-    __syncwarp();  // this step's counts before the next step's reads
+#pragma unroll
+    for (int u = 0; u < kSortBatch; ++u) {
+      const int f = b0 + 32 * u + lane;
+      int e = ev[u];
+      if (e >= E || (f < f1 && e < 0)) {
+        set_device_error(kErrExpertRange);
+        e = -1;
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0) my_cnt_row[e] += __popc(peers);
+      __syncwarp();  // this step's counts before the next step's reads
+    }
   }
   __syncthreads();
 
@@ -114,21 +125,30 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   }
   __syncthreads();
 
-  // 3. stable placement, each warp in its chunk's order
-  for (int b = f0; b < f1; b += 32) {
-    const int f = b + lane;
-    int e = f < f1 ? a.ids[f] : -1;
-    if (e >= E) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    const uint32_t lower = peers & ((1u << lane) - 1u);
-    int pos = 0;
-    if (e >= 0) pos = my_cnt_row[e] + __popc(lower);
-    __syncwarp();
-    if (e >= 0) {
-      a.sorted[pos] = f;
-      if (lower == 0) my_cnt_row[e] += __popc(peers);
+  // 3. stable placement, each warp in its chunk's order (ids batched as above)
+  for (int b0 = f0; b0 < f1; b0 += 32 * kSortBatch) {
+    int ev[kSortBatch];
+#pragma unroll
+    for (int u = 0; u < kSortBatch; ++u) {
+      const int f = b0 + 32 * u + lane;
+      ev[u] = f < f1 ? a.ids[f] : -1;
     }
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kSortBatch; ++u) {
+      const int f = b0 + 32 * u + lane;
+      int e = ev[u];
+      if (e >= E) e = -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const uint32_t lower = peers & ((1u << lane) - 1u);
+      int pos = 0;
+      if (e >= 0) pos = my_cnt_row[e] + __popc(lower);
+      __syncwarp();
+      if (e >= 0) {
+        a.sorted[pos] = f;
+        if (lower == 0) my_cnt_row[e] += __popc(peers);
+      }
+      __syncwarp();
+    }
   }
 }
 
