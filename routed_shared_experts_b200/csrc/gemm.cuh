@@ -58,18 +58,21 @@ __host__ __device__ constexpr bool is_mx(int kind) { return kind == kMx8 || kind
 // stage 2 at 128 tokens shares three accumulators between its two groups, the
 // scale ring taking TMEM's last columns.
 //
-// Copy issue: a thread needs about 130 cycles to issue one TMA copy, so at
-// 64-token tiles and more, where a stage holds a large token tile too, two
-// producer warps share it: warp 0 loads the weight tile (and its MX scale
-// tile), warp 2 the token tile (and its scale tile); both arm the stage's
-// `full` barrier with their own bytes. Smaller tiles keep one producer warp.
+// Copy issue: a thread needs about 130 cycles to issue one TMA copy, so where
+// a stage holds four copies (block-scaled kernels: two operand tiles and their
+// scale tiles) or a large token tile (64+ tokens), two producer warps share
+// them: warp 0 loads the weight tile (and its MX scale tile), warp 2 the token
+// tile (and its scale tile); both arm the stage's `full` barrier with their
+// own bytes. The block-scaled kernels also give the two TMEM copies of a
+// stage's scale tiles to warp 3, so that the MMA thread issues MMAs only.
 template <int BN, int KIND, bool S1>
 struct EpiCfg {
   static constexpr bool kMxWide = is_mx(KIND) && BN == 128 && !S1;
   static constexpr int kGroups = (is_mx(KIND) ? (BN <= 32 || !S1) : BN <= 128) ? 2 : 1;
   static constexpr int kAcc = kMxWide ? 3 : 2 * kGroups;
-  static constexpr bool kSplit = BN >= 64;              // two producer warps
-  static constexpr int kLead = kSplit ? 96 : 64;         // threads before the epilogue warps
+  static constexpr bool kSplit = BN >= 64 || is_mx(KIND);  // two producer warps
+  static constexpr bool kSfWarp = is_mx(KIND);               // warp 3 copies scale tiles (one-CTA tiles)
+  static constexpr int kLead = kSfWarp ? 128 : kSplit ? 96 : 64;  // threads before the epilogue warps
   static constexpr int kThreads = kLead + kEpiThreads * kGroups;
 };
 
@@ -121,8 +124,12 @@ struct GemmSmem {
   static constexpr int kSfBytes = kMx ? 2 * kSfTile : 0;  // A then B scale tile
   static constexpr int kStageBytes = kABytes + kBBytes + kSfBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  // full[S], empty[S], acc_full[A], acc_empty[A], drain
-  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1;
+  // scale tiles in TMEM: copied by warp 3 into slot `stage` (one-CTA tiles),
+  // else by the MMA thread into a ring of kSfSlots (pairs; warp 3 idles)
+  static constexpr bool kSfWarp = EpiCfg<BN, KIND, S1>::kSfWarp && !PAIR;
+  static constexpr int kSfRing = kSfWarp ? STAGES : kSfSlots;
+  // full[S], empty[S], acc_full[A], acc_empty[A], drain, then sf_full[S] with the scale-copy warp
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAcc + 1 + (kSfWarp ? STAGES : 0);
   static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
   // tmem slot, abort flag, grid-barrier flag, pad word; then per epilogue group: ok flag +
   // 3 pad words, tok[BN], wgt[BN], last[BN], amax_part[4][BN]
@@ -131,7 +138,7 @@ struct GemmSmem {
   static constexpr int kBytes = kMiscOffset + kMiscBytes + 1024;  // + alignment slack
   static constexpr int kAccCols = kAcc * BN;
   static constexpr int kSfCol = kAccCols;  // first column of the scale ring
-  static constexpr int kColsNeeded = kAccCols + (kMx ? 8 * kSfSlots : 0);
+  static constexpr int kColsNeeded = kAccCols + (kMx ? 8 * kSfRing : 0);
   static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 : kColsNeeded <= 128 ? 128
                                    : kColsNeeded <= 256 ? 256 : 512;
   static_assert(kColsNeeded <= 512, "TMEM");
@@ -473,6 +480,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
   constexpr int kMmaM = PAIR ? 2 * kTileM : kTileM;
   constexpr bool SPLIT = EpiCfg<BN, KIND, S1>::kSplit;
   constexpr int kLead = EpiCfg<BN, KIND, S1>::kLead;
+  constexpr bool SFW = L::kSfWarp;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
   static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
@@ -485,6 +493,7 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + NACC;
   uint64_t* drain = acc_empty + NACC;
+  uint64_t* sf_full = drain + 1;  // SFW: stage s's scale tiles are in TMEM slot s
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* group_base = reinterpret_cast<int*>(tmem_slot + 4);
@@ -506,6 +515,8 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
       mbar_init(&acc_empty[a], kAccEmptyCount);
     }
     mbar_init(drain, 1);
+    if constexpr (SFW)
+      for (int s = 0; s < STAGES; ++s) mbar_init(&sf_full[s], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -678,14 +689,17 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         if (ok) tc_fence_after();
         for (int kb = 0; ok && kb < g.num_kb; ++kb) {
-          ok = mbar_wait(&full[stage], phase, abort_flag);
+          ok = mbar_wait(SFW ? &sf_full[stage] : &full[stage], phase, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
           const uint64_t adesc = sw128_kmajor_desc(a_addr);
           const uint64_t bdesc = sw128_kmajor_desc(a_addr + L::kABytes);
           uint32_t tsfa = 0, tsfb = 0;
-          if (MX) {
+          if (SFW) {
+            tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol + 8 * stage);
+            tsfb = tsfa + 4;
+          } else if (MX) {
             // scale tiles of this stage -> TMEM ring slot (A: 4 columns, B: the next 4)
             tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol) + sf_slot * 8;
             tsfb = tsfa + 4;
@@ -747,6 +761,42 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
       else umma_commit(drain);
       drain_wait(drain, 0);
     }
+  } else if (SFW && warp == 3) {
+    // ------------------------------------------------------------ scale-tile copier
+    // Lane 0 copies each stage's A and B scale tiles into TMEM slot `stage`
+    // (columns kSfCol + 8 * stage, A then B) and commits the copies to
+    // sf_full[stage], which the MMA thread waits on in place of `full`. A slot
+    // needs no barrier of its own: stage s is refilled, and its `full` barrier
+    // completes again, only after the MMAs that read slot s have finished
+    // (the MMA thread's commit to empty[s]).
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int last = -1;  // stage of the last commit, drained on the way out
+      uint32_t last_phase = 0;
+      for (int tile = unit0; ok && tile < total; tile += n_units) {
+        for (int kb = 0; kb < g.num_kb; ++kb) {
+          ok = mbar_wait(&full[stage], phase, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sf_addr = smem_u32(smem + stage * L::kStageBytes) + L::kABytes + L::kBBytes;
+          const uint32_t tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol + 8 * stage);
+          tmem_cp_32x128b_x4(tsfa, plain_rows16_desc(sf_addr));
+          tmem_cp_32x128b_x4(tsfa + 4, plain_rows16_desc(sf_addr + kSfTile));
+          umma_commit(&sf_full[stage]);
+          last = stage;
+          last_phase = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // every copy issued (the last commit tracks all of them) lands before TMEM is freed
+      if (last >= 0) drain_wait(&sf_full[last], last_phase);
+    }
+    __syncwarp();
   } else if (warp >= kLead / 32) {
     // ------------------------------------------------------------ epilogue
     const int grp = (warp - kLead / 32) >> 2;     // epilogue group: tiles j with j % G == grp
