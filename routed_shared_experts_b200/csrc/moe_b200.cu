@@ -109,15 +109,23 @@ moe_status_t make_sf_tile_map(CUtensorMap* m, const void* base, size_t tiles) {
 
 // ------------------------------------------------------------ GEMM dispatch
 
-template <int BN, int KIND>
+template <int BN, int KIND, bool S1, int ST = 2>
+constexpr int fit_stages() {
+  if constexpr (ST < 16 && moe::GemmSmem<BN, ST + 1, KIND, S1>::kBytes <= 227 * 1024)
+    return fit_stages<BN, KIND, S1, ST + 1>();
+  else
+    return ST;
+}
+
+template <int BN, int KIND, bool S1>
 constexpr int stages_for() {
   // as many stages as fit in 227 KB of shared memory, one CTA per SM, except
   // bf16 / fp8 16-token tiles: six stages (108 KB of operands in flight per SM)
   // streamed the weights faster than twelve (decode step 152.3 -> 150.4 us
   // bf16, 194.5 -> 182.6 us fp8 at T = 32), as a bulk-copy stream also peaks at
   // 64-100 KB in flight per SM and loses DRAM bandwidth beyond
-  if (moe::is_mx(KIND)) return BN == 16 ? 11 : BN == 32 ? 10 : BN == 64 ? 8 : 6;
-  return BN == 16 ? 6 : BN == 32 ? 11 : BN == 64 ? 9 : BN == 128 ? 6 : 4;
+  if constexpr (!moe::is_mx(KIND) && BN == 16) return 6;
+  else return fit_stages<BN, KIND, S1>();
 }
 
 // Pair tiles: as many stages as fit in 227 KB (each CTA holds half the token rows).
@@ -160,7 +168,7 @@ moe_status_t set_smem_attr(Kern kern, int bytes, std::atomic<int>* attr_set) {
 template <int BN, bool S1, int KIND>
 moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb16,
                             const moe::GemmArgs& g, int max_tiles, cudaStream_t s) {
-  constexpr int ST = stages_for<BN, KIND>();
+  constexpr int ST = stages_for<BN, KIND, S1>();
   using L = moe::GemmSmem<BN, ST, KIND, S1>;
   static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
   auto kern = moe::k_moe_gemm<BN, ST, S1, KIND, false>;
