@@ -246,7 +246,10 @@ moe_status_t moe_router_gemm_topk(int dtype, const void* x, const void* w_r, con
  *   expert_counts int32 [E]; expert_offsets int32 [E+1] (padded prefix sum);
  *   num_padded    int32 [1] = expert_offsets[E].
  * Checks: block_m in {16,32,64,128,256}; T*k <= 1<<20; E <= MOE_MAX_EXPERTS.
- * An expert id outside [0,E) sets device error 2 and is dropped. */
+ * An expert id outside [0,E) sets device error 2 and is dropped.
+ * One CTA of 1024 threads below 4096 slots; from 4096 on, a cluster of 8 such
+ * CTAs, each sorting its eighth of the slots and reading the others' per-expert
+ * counts over distributed shared memory (the results are the same). */
 moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
                             int32_t* sorted_ids, int32_t* block_expert, int32_t* expert_counts,
                             int32_t* expert_offsets, int32_t* num_padded, moe_stream_t stream);

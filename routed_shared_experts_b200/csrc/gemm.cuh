@@ -79,16 +79,17 @@ struct EpiCfg {
 // 128-byte K atoms (one swizzle row of every operand row) per pipeline stage.
 // Every stage costs each role a fixed amount of issue - a barrier wait, an
 // expect-tx arrival, a commit, the loop: 200-500 cycles per role, measured -
-// besides its copies and MMAs. Where those fixed costs set the pace (64- and
-// 128-token tiles; the block-scaled kernels, whose stages carry two more
-// copies and two scale-tile moves, at every tile size) a stage carries two
-// atoms: two copies per operand into consecutive swizzle blocks, one
-// scale-tile copy per operand for both. Measured against one atom per stage:
-// MXFP8 prefill layer 5178 -> 4278 us, MXFP4 prefill 4810 -> 3705 us, fp8
-// a8w8 506 -> 416 us, MXFP4 decode 101.6 -> 88.6 us.
+// besides its copies and MMAs, and those fixed costs set the pace of these
+// kernels. So a stage carries two atoms (two copies per operand into
+// consecutive swizzle blocks, one scale-tile copy per operand for both, eight
+// MMAs per barrier round trip). Measured against one atom per stage: MXFP8
+// prefill layer 5178 -> 4278 us, MXFP4 prefill 4810 -> 3705 us, fp8 a8w8
+// 506 -> 416 us, MXFP4 decode 101.6 -> 88.6 us, bf16 decode 150.1 -> 145.5
+// us, fp8 decode (T = 32) 181.8 -> 177.8 us. 256-token tiles (and pairs)
+// keep one atom: two would leave two stages of shared memory.
 template <int BN, int KIND, bool PAIR>
 __host__ __device__ constexpr int atoms_for() {
-  return (!PAIR && ((BN >= 64 && BN <= 128) || is_mx(KIND))) ? 2 : 1;
+  return (!PAIR && BN <= 128) ? 2 : 1;
 }
 
 struct GemmArgs {

@@ -120,11 +120,12 @@ constexpr int fit_stages() {
 template <int BN, int KIND, bool S1>
 constexpr int stages_for() {
   // as many stages as fit in 227 KB of shared memory, one CTA per SM, except
-  // bf16 / fp8 16-token tiles: six stages (108 KB of operands in flight per SM)
-  // streamed the weights faster than twelve (decode step 152.3 -> 150.4 us
-  // bf16, 194.5 -> 182.6 us fp8 at T = 32), as a bulk-copy stream also peaks at
-  // 64-100 KB in flight per SM and loses DRAM bandwidth beyond
-  if constexpr (!moe::is_mx(KIND) && BN == 16) return 6;
+  // bf16 / fp8 16-token tiles: 108 KB of operands in flight per SM (three
+  // two-atom stages) streamed the weights faster than all that fit (decode
+  // step 145.5 us either way for bf16, 177.8 against 193.5 us for fp8 at
+  // T = 32), as a bulk-copy stream also peaks at 64-100 KB in flight per SM
+  // and loses DRAM bandwidth beyond
+  if constexpr (!moe::is_mx(KIND) && BN == 16) return 3;
   else return fit_stages<BN, KIND, S1>();
 }
 
@@ -527,16 +528,22 @@ moe_status_t moe_align_sort(const int32_t* topk_ids, int T, int top_k, int E, in
   if (static_cast<long long>(T) * top_k > (1ll << 20)) return MOE_ERR_SHAPE;
   moe::SortArgs a{topk_ids, T * top_k, E, block_m, sorted_ids, block_expert, expert_counts, expert_offsets,
                   num_padded};
-  const size_t smem = (2 * static_cast<size_t>(E) + 32 * static_cast<size_t>(E) + 32) * sizeof(int);
-  static std::atomic<int> attr_set[64];
-  int dev = 0;
-  MOE_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64 || !attr_set[dev].load()) {
-    MOE_CK(cudaFuncSetAttribute(moe::k_align_sort, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>((2 + 32) * MOE_MAX_EXPERTS * sizeof(int) + 32 * sizeof(int))));
-    if (dev >= 0 && dev < 64) attr_set[dev].store(1);
+  const size_t smem = moe::sort_smem_bytes(E);
+  const int smem_max = static_cast<int>(moe::sort_smem_bytes(MOE_MAX_EXPERTS));
+  // a cluster of CTAs from kSortClusterMinSlots slots on (one CTA's 32 warps
+  // take 32-slot steps one after another; the cluster splits them 8 ways)
+  const bool cluster = a.N >= moe::kSortClusterMinSlots;
+  if (cluster) {
+    static std::atomic<int> attr_set[64];
+    const moe_status_t r = set_smem_attr(moe::k_align_sort_cluster, smem_max, attr_set);
+    if (r != MOE_OK) return r;
+    moe::k_align_sort_cluster<<<moe::kSortCluster, moe::kSortThreads, smem, as_stream(stream)>>>(a);
+  } else {
+    static std::atomic<int> attr_set[64];
+    const moe_status_t r = set_smem_attr(moe::k_align_sort, smem_max, attr_set);
+    if (r != MOE_OK) return r;
+    moe::k_align_sort<<<1, moe::kSortThreads, smem, as_stream(stream)>>>(a);
   }
-  moe::k_align_sort<<<1, moe::kSortThreads, smem, as_stream(stream)>>>(a);
   MOE_CK(cudaGetLastError());
   return MOE_OK;
 }

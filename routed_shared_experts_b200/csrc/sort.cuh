@@ -1,4 +1,5 @@
-// sort.cuh - align/sort of the routed slots by expert, one CTA of 32 warps.
+// sort.cuh - align/sort of the routed slots by expert: one CTA of 32 warps
+// for small batches, a cluster of kSortCluster such CTAs for large ones.
 //
 // vllm-project/vllm PR 65207, reviewer measurements ("Commits 2 and 3"):
 // moe_sorting is run without zeroing the layer output; here the sort never
@@ -10,7 +11,9 @@
 namespace moe {
 
 constexpr int kSortThreads = 1024;
-constexpr int kSortBatch = 8;  // 32-slot steps whose ids a warp loads at once
+constexpr int kSortCluster = 8;              // CTAs of the cluster sort
+constexpr int kSortClusterMinSlots = 4096;   // slots from which the cluster sort runs
+constexpr int kSortClusterBatch = 4;         // id loads per warp in flight (cluster sort)
 
 struct SortArgs {
   const int32_t* ids;  // [N] flat slots f = t*k + j
@@ -22,52 +25,42 @@ struct SortArgs {
   int32_t* num_padded;    // [1]
 };
 
-// Shared memory: cnt[E], base[E], warp_cnt[32][E], warp totals [32].
-//
-// Each warp owns one contiguous chunk of the flat slots (warp w: chunk w of
-// 32), so that a stable order needs no barrier per round:
-//   1. each warp counts its chunk's slots per expert into its own row of
+// Shared memory of either kernel: tot[E], base[E], warp_cnt[32][E], warp sums [32].
+__host__ __device__ constexpr size_t sort_smem_bytes(int E) {
+  return (2 * static_cast<size_t>(E) + 32 * static_cast<size_t>(E) + 32) * sizeof(int);
+}
+
+// Each warp owns one contiguous range [f0, f1) of the flat slots, so that a
+// stable order needs no barrier per round:
+//   1. the warp counts its range's slots per expert into its own row of
 //      warp_cnt (32 slots per step, __match_any_sync groups equal experts, the
 //      lowest lane of a group adds the group's size: one writer per entry);
-//   2. per expert, an exclusive prefix over the 32 warps' counts, and over
-//      the experts an exclusive prefix of the padded segment sizes, turn each
-//      warp_cnt entry into the absolute position of that warp's first slot of
-//      that expert; counts, offsets, block owners and padding are written;
-//   3. each warp walks its chunk again in order and places every slot at its
+//   2. exclusive prefixes - over the warps (and, in the cluster sort, over the
+//      CTAs before this one) per expert, and over the experts' padded segment
+//      sizes - turn each warp_cnt entry into the absolute position of that
+//      warp's first slot of that expert; counts, offsets, block owners and
+//      padding are written once;
+//   3. the warp walks its range again in order and places every slot at its
 //      entry plus its rank among the equal experts of its 32-slot step, then
 //      advances the entry: ascending f inside every expert segment.
-__global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
-  extern __shared__ int ssm[];
-  const int E = a.E;
-  int* cnt = ssm;
-  int* base = cnt + E;
-  int* warp_cnt = base + E;
-  int* wsum = warp_cnt + 32 * E;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int chunk = (a.N + 31) / 32;
-  const int f0 = warp * chunk;
-  const int f1 = f0 + chunk < a.N ? f0 + chunk : a.N;
-  int* my_cnt_row = warp_cnt + warp * E;
-
-  for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
-  __syncthreads();
-
-  // 1. per-warp counts; the ids of kSortBatch steps are loaded before any is
-  // used, so that a warp keeps that many loads in flight
-  for (int b0 = f0; b0 < f1; b0 += 32 * kSortBatch) {
-    int ev[kSortBatch];
+// B: 32-slot steps whose ids a warp loads before it uses any (B loads in
+// flight instead of one per step; the single-CTA sort of small batches,
+// whose warps take a step or two, is fastest with B = 1).
+template <int B>
+__device__ __forceinline__ void sort_count(const SortArgs& a, int f0, int f1, int* my_cnt_row) {
+  const int lane = threadIdx.x & 31;
+  for (int b0 = f0; b0 < f1; b0 += 32 * B) {
+    int ev[B];
 #pragma unroll
-    for (int u = 0; u < kSortBatch; ++u) {
+    for (int u = 0; u < B; ++u) {
       const int f = b0 + 32 * u + lane;
       ev[u] = f < f1 ? a.ids[f] : -1;
     }
 #pragma unroll
-    for (int u = 0; u < kSortBatch; ++u) {
+    for (int u = 0; u < B; ++u) {
       const int f = b0 + 32 * u + lane;
       int e = ev[u];
-      if (e >= E || (f < f1 && e < 0)) {
+      if (e >= a.E || (f < f1 && e < 0)) {
         set_device_error(kErrExpertRange);
         e = -1;
       }
@@ -76,68 +69,23 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
       __syncwarp();  // this step's counts before the next step's reads
     }
   }
-  __syncthreads();
+}
 
-  // 2. exclusive prefix over warps (per expert), then over padded segments
-  int my_cnt = 0;
-  if (tid < E) {
-    int run = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int c = warp_cnt[w * E + tid];
-      warp_cnt[w * E + tid] = run;
-      run += c;
-    }
-    my_cnt = run;
-    cnt[tid] = run;
-  }
-  const int my_pad = tid < E ? (my_cnt + a.bm - 1) / a.bm * a.bm : 0;
-  int incl = my_pad;
+template <int B>
+__device__ __forceinline__ void sort_place(const SortArgs& a, int f0, int f1, int* my_cnt_row) {
+  const int lane = threadIdx.x & 31;
+  for (int b0 = f0; b0 < f1; b0 += 32 * B) {
+    int ev[B];
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int v = wsum[lane];
-    int s = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += o;
-    }
-    wsum[lane] = s - v;  // exclusive over warps
-  }
-  __syncthreads();
-  const int excl = incl - my_pad + wsum[warp];
-  if (tid < E) {
-    base[tid] = excl;
-    a.counts[tid] = my_cnt;
-    a.offsets[tid] = excl;
-    if (tid == E - 1) {
-      a.offsets[E] = excl + my_pad;
-      *a.num_padded = excl + my_pad;
-    }
-    for (int b = excl / a.bm; b < (excl + my_pad) / a.bm; ++b) a.block_expert[b] = tid;
-    for (int p = excl + my_cnt; p < excl + my_pad; ++p) a.sorted[p] = a.N;  // sentinel
-    for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += excl;  // absolute start of warp w's slots of tid
-  }
-  __syncthreads();
-
-  // 3. stable placement, each warp in its chunk's order (ids batched as above)
-  for (int b0 = f0; b0 < f1; b0 += 32 * kSortBatch) {
-    int ev[kSortBatch];
-#pragma unroll
-    for (int u = 0; u < kSortBatch; ++u) {
+    for (int u = 0; u < B; ++u) {
       const int f = b0 + 32 * u + lane;
       ev[u] = f < f1 ? a.ids[f] : -1;
     }
 #pragma unroll
-    for (int u = 0; u < kSortBatch; ++u) {
+    for (int u = 0; u < B; ++u) {
       const int f = b0 + 32 * u + lane;
       int e = ev[u];
-      if (e >= E) e = -1;
+      if (e >= a.E) e = -1;
       const uint32_t peers = __match_any_sync(0xffffffffu, e);
       const uint32_t lower = peers & ((1u << lane) - 1u);
       int pos = 0;
@@ -150,6 +98,147 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
       __syncwarp();
     }
   }
+}
+
+// Per expert e = threadIdx.x < E: warp_cnt[w][e] becomes the exclusive prefix
+// over warps; returns this CTA's count of e (0 for other threads).
+__device__ __forceinline__ int sort_warp_prefix(int* warp_cnt, int E) {
+  const int tid = threadIdx.x;
+  int run = 0;
+  if (tid < E) {
+    for (int w = 0; w < 32; ++w) {
+      const int c = warp_cnt[w * E + tid];
+      warp_cnt[w * E + tid] = run;
+      run += c;
+    }
+  }
+  return run;
+}
+
+// Exclusive prefix over experts of the padded segment sizes (block-wide;
+// every thread calls it); returns expert tid's segment start.
+__device__ __forceinline__ int sort_segment_prefix(int my_pad, int* wsum) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int incl = my_pad;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = wsum[lane];
+    int s = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += o;
+    }
+    wsum[lane] = s - v;  // exclusive over warps
+  }
+  __syncthreads();
+  return incl - my_pad + wsum[warp];
+}
+
+// Expert tid's outputs: count, offset, block owners, sentinel padding.
+__device__ __forceinline__ void sort_write_segment(const SortArgs& a, int e, int cnt, int excl, int pad) {
+  a.counts[e] = cnt;
+  a.offsets[e] = excl;
+  if (e == a.E - 1) {
+    a.offsets[a.E] = excl + pad;
+    *a.num_padded = excl + pad;
+  }
+  for (int b = excl / a.bm; b < (excl + pad) / a.bm; ++b) a.block_expert[b] = e;
+  for (int p = excl + cnt; p < excl + pad; ++p) a.sorted[p] = a.N;  // sentinel
+}
+
+// One CTA: warp w owns chunk w of 32 equal chunks of the slots.
+__global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
+  extern __shared__ int ssm[];
+  const int E = a.E;
+  int* warp_cnt = ssm + 2 * E;
+  int* wsum = warp_cnt + 32 * E;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int chunk = (a.N + 31) / 32;
+  const int f0 = warp * chunk;
+  const int f1 = f0 + chunk < a.N ? f0 + chunk : a.N;
+  int* my_cnt_row = warp_cnt + warp * E;
+
+  for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
+  __syncthreads();
+  sort_count<1>(a, f0, f1, my_cnt_row);
+  __syncthreads();
+  const int cnt = sort_warp_prefix(warp_cnt, E);
+  const int pad = tid < E ? (cnt + a.bm - 1) / a.bm * a.bm : 0;
+  const int excl = sort_segment_prefix(pad, wsum);
+  if (tid < E) {
+    sort_write_segment(a, tid, cnt, excl, pad);
+    for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += excl;  // absolute start of warp w's slots of tid
+  }
+  __syncthreads();
+  sort_place<1>(a, f0, f1, my_cnt_row);
+}
+
+// kSortCluster CTAs: CTA r owns part r of kSortCluster equal parts of the
+// slots, its warps 32 equal chunks of that part. After each CTA's counts, a
+// cluster barrier makes every CTA's per-expert totals readable over
+// distributed shared memory; each CTA adds up, per expert, the totals of all
+// CTAs (the segment sizes, identical in every CTA) and of the CTAs before it
+// (its start inside the segment). CTA 0 writes the segment outputs. A second
+// cluster barrier, arrived at once the totals are read and waited on at the
+// end, keeps every CTA's shared memory alive until the others have read it.
+__global__ void __cluster_dims__(kSortCluster, 1, 1) __launch_bounds__(kSortThreads)
+    k_align_sort_cluster(const SortArgs a) {
+  extern __shared__ int ssm[];
+  const int E = a.E;
+  int* tot = ssm;  // this CTA's count of each expert, read by the cluster
+  int* warp_cnt = ssm + 2 * E;
+  int* wsum = warp_cnt + 32 * E;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int part = (a.N + kSortCluster - 1) / kSortCluster;
+  const int p0 = rank * part < a.N ? rank * part : a.N;
+  const int p1 = p0 + part < a.N ? p0 + part : a.N;
+  const int chunk = (p1 - p0 + 31) / 32;
+  const int f0 = p0 + warp * chunk < p1 ? p0 + warp * chunk : p1;
+  const int f1 = f0 + chunk < p1 ? f0 + chunk : p1;
+  int* my_cnt_row = warp_cnt + warp * E;
+
+  for (int i = tid; i < 32 * E; i += kSortThreads) warp_cnt[i] = 0;
+  __syncthreads();
+  sort_count<kSortClusterBatch>(a, f0, f1, my_cnt_row);
+  __syncthreads();
+  const int mine = sort_warp_prefix(warp_cnt, E);
+  if (tid < E) tot[tid] = mine;
+  cluster_sync_all();  // every CTA's totals written and visible
+  int cnt = 0, before = 0;
+  if (tid < E) {
+    // every remote load issued before any is used
+    const uint32_t addr = smem_u32(tot + tid);
+    int c[kSortCluster];
+#pragma unroll
+    for (int r = 0; r < kSortCluster; ++r) c[r] = ld_shared_cluster_s32(mapa_shared(addr, static_cast<uint32_t>(r)));
+#pragma unroll
+    for (int r = 0; r < kSortCluster; ++r) {
+      if (r < rank) before += c[r];
+      cnt += c[r];
+    }
+  }
+  cluster_arrive_release();  // this CTA has read every other CTA's totals
+  const int pad = tid < E ? (cnt + a.bm - 1) / a.bm * a.bm : 0;
+  const int excl = sort_segment_prefix(pad, wsum);
+  if (tid < E) {
+    if (rank == 0) sort_write_segment(a, tid, cnt, excl, pad);
+    const int start = excl + before;
+    for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += start;
+  }
+  __syncthreads();
+  sort_place<kSortClusterBatch>(a, f0, f1, my_cnt_row);
+  cluster_wait_acquire();  // no CTA leaves while another may still read its totals
 }
 
 }  // namespace moe

@@ -96,16 +96,24 @@ def _sort_gpu(ids_np, E, bm):
         int(num_padded.item())
 
 
+# T*k below and from 4096 slots on (one CTA / the 8-CTA cluster sort),
+# including exactly 4095 and 4096, a ragged last cluster part, E = 512 and
+# the largest batch the call accepts (T*k = 2^20)
 @pytest.mark.parametrize("T,k,E,bm,skew", [(16, 2, 8, 16, 0), (32, 8, 128, 16, 0), (1024, 6, 64, 128, 0),
                                            (4096, 8, 256, 128, 1), (1, 1, 1, 16, 0), (3, 1, 512, 256, 0),
-                                           (2000, 4, 16, 32, 1), (128, 6, 64, 16, 0), (5, 3, 7, 64, 0)])
+                                           (2000, 4, 16, 32, 1), (128, 6, 64, 16, 0), (5, 3, 7, 64, 0),
+                                           (4095, 1, 33, 16, 0), (512, 8, 512, 64, 1), (8191, 2, 300, 256, 1),
+                                           (131072, 8, 256, 128, 1)])
 def test_align_sort_bit_exact(cuda_lib, T, k, E, bm, skew):
     rng = np.random.default_rng(T + E + bm)
     p = None
     if skew:
         p = 1.0 / np.arange(1, E + 1) ** 1.2
         p /= p.sum()
-    ids = np.stack([rng.choice(E, k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    if T * k > 100000:  # distinct experts per token do not matter to the sort
+        ids = rng.choice(E, size=(T, k), p=p).astype(np.int32)
+    else:
+        ids = np.stack([rng.choice(E, k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
     s, be, c, o, n = _sort_gpu(ids, E, bm)
     ref = oracle.align_sort(ids, E, bm)
     assert n == ref["num_padded"]
@@ -121,6 +129,21 @@ def test_align_sort_rejects_bad_ids(cuda_lib):
     s, be, c, o, n = _sort_gpu(ids, 4, 16)
     assert capi.device_error() == 2
     assert c.sum() == 3
+
+
+def test_align_sort_cluster_rejects_bad_ids(cuda_lib):
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, 64, size=(1024, 8)).astype(np.int32)
+    ids[700, 3] = 64  # out of range for E = 64
+    ids[1000, 0] = -1
+    s, be, c, o, n = _sort_gpu(ids, 64, 128)
+    assert capi.device_error() == 2
+    assert c.sum() == ids.size - 2
+    flat = ids.reshape(-1)
+    ok = (flat >= 0) & (flat < 64)
+    assert np.array_equal(c, np.bincount(flat[ok], minlength=64))
+    for e in range(64):  # every valid slot in its expert's segment, ascending; the two bad ones nowhere
+        assert np.array_equal(s[o[e]:o[e] + c[e]], np.nonzero(flat == e)[0])
 
 
 def _ulp(v, dt):
