@@ -40,14 +40,14 @@
  *     records a code in a device error word read by moe_device_error().
  *   - Layouts are row-major and dense unless stated. T tokens, H hidden, E
  *     routed experts, k = top_k, I expert intermediate size.
- *   - With MOE_B200_PAIR=1 in the environment, the grouped GEMMs of 128-token
- *     blocks run on CTA pairs (2-CTA clusters sharing one M = 256 tensor-core
- *     MMA, each SM loading its 128 weight rows and half of the token rows)
- *     when the weight rows split into an even number of 128-row tiles (stage
- *     1: I % 128 == 0, except the fp8 stage 1, whose per-row quantisation
- *     follows a grid barrier; stage 2: H % 256 == 0); by default one CTA per
- *     tile (measured a few percent faster). Results do not depend on the
- *     choice.
+ *   - With MOE_B200_PAIR=1 in the environment, the grouped GEMMs of 16- and
+ *     128-token blocks run on CTA pairs (2-CTA clusters sharing one M = 256
+ *     tensor-core MMA, each SM loading its 128 weight rows and half of the
+ *     token rows) when the weight rows split into an even number of 128-row
+ *     tiles (stage 1: I % 128 == 0, except the fp8 stage 1, whose per-row
+ *     quantisation follows a grid barrier; stage 2: H % 256 == 0); by default
+ *     one CTA per tile (measured faster on every workload but fp8 decode).
+ *     Results do not depend on the choice.
  *   - Shapes the grouped GEMMs cover (anything else returns MOE_ERR_SHAPE or
  *     MOE_ERR_ALIGNMENT and launches nothing): H % 128 == 0 (stage 1 with bf16
  *     operands: H % 64 == 0), I % 64 == 0, and I % 128 == 0 for MXFP8 and

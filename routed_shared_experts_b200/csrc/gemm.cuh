@@ -85,11 +85,11 @@ struct EpiCfg {
 // MMAs per barrier round trip). Measured against one atom per stage: MXFP8
 // prefill layer 5178 -> 4278 us, MXFP4 prefill 4810 -> 3705 us, fp8 a8w8
 // 506 -> 416 us, MXFP4 decode 101.6 -> 88.6 us, bf16 decode 150.1 -> 145.5
-// us, fp8 decode (T = 32) 181.8 -> 177.8 us. 256-token tiles (and pairs)
-// keep one atom: two would leave two stages of shared memory.
+// us, fp8 decode (T = 32) 181.8 -> 177.8 us. 256-token tiles keep one atom:
+// two would leave two stages of shared memory.
 template <int BN, int KIND, bool PAIR>
 __host__ __device__ constexpr int atoms_for() {
-  return (!PAIR && BN <= 128) ? 2 : 1;
+  return BN <= 128 ? 2 : 1;
 }
 
 struct GemmArgs {
@@ -503,7 +503,6 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
   constexpr int kLead = EpiCfg<BN, KIND, S1>::kLead;
   constexpr bool SFW = L::kSfWarp;
   constexpr int KA = L::kAtoms;
-  static_assert(!PAIR || KA == 1, "pair stages hold one K atom");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "token tile");
   static_assert(!MX || BN <= 128, "MXFP8 scale tiles cover 128 token rows");
   static_assert(STAGES <= 32, "stage mask");
@@ -622,15 +621,24 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
           if (lane == 0) {
             pending &= ~(1u << stage);
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);  // both CTAs' copies of this kind
-            if (do_w) {
-              if (S1) tma_load_5d_pair(a_dst, &tmA, fb, kb0 * KE, 0, 0, mt * 4, expert, pol_w);
-              else tma_load_3d_pair(a_dst, &tmA, fb, kb0 * KE, mt * kTileM, expert, pol_w);
-              if (MX) tma_load_2d_pair(sfa_dst, &tmSfa, fb, 0, ((expert * g.n_mt + mt) * g.num_kb + kb0) * 4, pol_w);
-            }
-            if (do_t) {
-              if (ncols == BN) tma_load_2d_pair(b_dst, &tmB, fb, kb0 * KE, row0, pol_x);
-              if (MX) tma_load_2d_pair(sfb_dst, &tmSfb, fb, 0, (blk * g.num_kb + kb0) * 4, pol_x);
+            // both CTAs' copies of this kind, per atom
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes * static_cast<uint32_t>(na));
+#pragma unroll
+            for (int a = 0; a < KA; ++a) {
+              if (a >= na) break;
+              const int kb = kb0 + a;
+              if (do_w) {
+                uint8_t* dst = a_dst + a * L::kAtomA;
+                if (S1) tma_load_5d_pair(dst, &tmA, fb, kb * KE, 0, 0, mt * 4, expert, pol_w);
+                else tma_load_3d_pair(dst, &tmA, fb, kb * KE, mt * kTileM, expert, pol_w);
+                if (MX)
+                  tma_load_2d_pair(sfa_dst + a * kSfTile, &tmSfa, fb, 0, ((expert * g.n_mt + mt) * g.num_kb + kb) * 4,
+                                   pol_w);
+              }
+              if (do_t) {
+                if (ncols == BN) tma_load_2d_pair(b_dst + a * L::kAtomB, &tmB, fb, kb * KE, row0, pol_x);
+                if (MX) tma_load_2d_pair(sfb_dst + a * kSfTile, &tmSfb, fb, 0, (blk * g.num_kb + kb) * 4, pol_x);
+              }
             }
             pending |= 1u << stage;
             pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
@@ -638,8 +646,13 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
           if (!solo) __syncwarp();
           // a short tile: this CTA's token rows in 8-row boxes, issued by the lanes
           if (do_t && ncols < BN) {
-            for (int q = lane; q < my_rows / 8; q += 32)
-              tma_load_2d_pair(b_dst + q * 8 * kTileKBytes, &tmB16, fb, kb0 * KE, row0 + q * 8, pol_x);
+            const int boxes = my_rows / 8;  // per atom
+            for (int q = lane; q < na * boxes; q += 32) {
+              const int a = q / boxes;
+              const int r = q - a * boxes;
+              tma_load_2d_pair(b_dst + a * L::kAtomB + r * 8 * kTileKBytes, &tmB16, fb, (kb0 + a) * KE, row0 + r * 8,
+                               pol_x);
+            }
           }
         } else {
           if (lane == 0) {
@@ -746,16 +759,21 @@ __global__ void __launch_bounds__(EpiCfg<BN, KIND, S1>::kThreads, 1)
             tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol + 8 * KA * stage);
             tsfb = tsfa + 4 * KA;
           } else if (MX) {
-            // scale tiles of this stage -> TMEM ring slot (A: 4 columns, B: the next 4)
-            tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol) + sf_slot * 8;
-            tsfb = tsfa + 4;
+            // scale tiles of this stage -> TMEM ring slot (the atoms' A tiles in
+            // 4 columns each, then their B tiles)
+            tsfa = tmem_base + static_cast<uint32_t>(L::kSfCol) + sf_slot * 8 * KA;
+            tsfb = tsfa + 4 * KA;
             const uint32_t sf_addr = a_addr + L::kABytes + L::kBBytes;
-            if constexpr (PAIR) {
-              tmem_cp_32x128b_x4_pair(tsfa, plain_rows16_desc(sf_addr));
-              tmem_cp_32x128b_x4_pair(tsfb, plain_rows16_desc(sf_addr + kSfTile));
-            } else {
-              tmem_cp_32x128b_x4(tsfa, plain_rows16_desc(sf_addr));
-              tmem_cp_32x128b_x4(tsfb, plain_rows16_desc(sf_addr + kSfTile));
+#pragma unroll
+            for (int a = 0; a < KA; ++a) {
+              if (a >= na) break;
+              if constexpr (PAIR) {
+                tmem_cp_32x128b_x4_pair(tsfa + 4 * a, plain_rows16_desc(sf_addr + a * kSfTile));
+                tmem_cp_32x128b_x4_pair(tsfb + 4 * a, plain_rows16_desc(sf_addr + (KA + a) * kSfTile));
+              } else {
+                tmem_cp_32x128b_x4(tsfa + 4 * a, plain_rows16_desc(sf_addr + a * kSfTile));
+                tmem_cp_32x128b_x4(tsfb + 4 * a, plain_rows16_desc(sf_addr + (KA + a) * kSfTile));
+              }
             }
             sf_slot = (sf_slot + 1) % kSfSlots;
           }

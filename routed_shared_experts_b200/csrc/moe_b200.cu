@@ -140,19 +140,19 @@ constexpr int pair_stages() {
 
 // Whether a GEMM runs on CTA pairs (one MMA of M = 256 per 2-CTA cluster,
 // each SM loading its 128 weight rows and half the token tile): opt-in with
-// MOE_B200_PAIR=1, for 128-token tiles whose weight rows split into an even
-// number of 128-row tiles, never the fp8 stage 1 (its per-row quantisation of
-// h follows a grid barrier in a cooperative launch). Measured on the prefill
-// layers, the pairs run a few percent slower than one CTA per tile: each
-// stage costs about the same number of issued copies per SM either way, and
-// the issue of copies and MMAs, not the operand bytes, paces these kernels.
-// Results do not depend on the choice.
+// MOE_B200_PAIR=1, for 16- and 128-token tiles whose weight rows split into
+// an even number of 128-row tiles, never the fp8 stage 1 (its per-row
+// quantisation of h follows a grid barrier in a cooperative launch). Measured
+// against one CTA per tile (two-atom stages both): MXFP8 prefill 4104 -> 4189
+// us, bf16 decode 143.3 -> 146.8 us, MXFP4 decode 87.2 -> 105.1 us (a pair's
+// MMA thread also moves the scale tiles), fp8 decode (T = 32) 175.3 -> 172.8
+// us. Results do not depend on the choice.
 bool use_pair(int dtype, int bm, int n_mt, bool s1) {
   static const bool enabled = [] {
     const char* v = getenv("MOE_B200_PAIR");
     return v && v[0] == '1';
   }();
-  return enabled && bm == 128 && n_mt % 2 == 0 && !(s1 && dtype == MOE_DT_FP8_E4M3);
+  return enabled && (bm == 16 || bm == 128) && n_mt % 2 == 0 && !(s1 && dtype == MOE_DT_FP8_E4M3);
 }
 
 template <typename Kern>
@@ -194,11 +194,10 @@ moe_status_t launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const 
 
 // A GEMM on CTA pairs: 2-CTA clusters, as many as can be resident at once
 // (cudaOccupancyMaxActiveClusters), each looping over pair tiles.
-template <bool S1, int KIND>
+template <int BN, bool S1, int KIND>
 moe_status_t launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb8,
                               const CUtensorMap& tsfa, const CUtensorMap& tsfb, const moe::GemmArgs& g,
                               int max_pair_tiles, cudaStream_t s) {
-  constexpr int BN = 128;
   constexpr int ST = pair_stages<BN, KIND, S1>();
   using L = moe::GemmSmem<BN, ST, KIND, S1, true>;
   static_assert(L::kBytes <= 227 * 1024, "shared memory per CTA");
@@ -264,16 +263,28 @@ moe_status_t launch_gemm_kind(int dtype, int bm, const CUtensorMap& ta, const CU
   return launch_gemm<S1, moe::kBf16>(bm, ta, tb, tb16, g, max_tiles, s);
 }
 
-template <bool S1>
-moe_status_t launch_gemm_pair_kind(int dtype, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb8,
-                                   const CUtensorMap& tsfa, const CUtensorMap& tsfb, const moe::GemmArgs& g,
-                                   int max_pair_tiles, cudaStream_t s) {
-  if (dtype == MOE_DT_MXFP8_E4M3) return launch_gemm_pair<S1, moe::kMx8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
-  if (dtype == MOE_DT_MXFP4_E2M1) return launch_gemm_pair<S1, moe::kMx4>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+template <int BN, bool S1>
+moe_status_t launch_gemm_pair_bn(int dtype, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb8,
+                                 const CUtensorMap& tsfa, const CUtensorMap& tsfb, const moe::GemmArgs& g,
+                                 int max_pair_tiles, cudaStream_t s) {
+  if (dtype == MOE_DT_MXFP8_E4M3)
+    return launch_gemm_pair<BN, S1, moe::kMx8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  if (dtype == MOE_DT_MXFP4_E2M1)
+    return launch_gemm_pair<BN, S1, moe::kMx4>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
   if constexpr (!S1) {
-    if (dtype == MOE_DT_FP8_E4M3) return launch_gemm_pair<S1, moe::kFp8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+    if (dtype == MOE_DT_FP8_E4M3)
+      return launch_gemm_pair<BN, S1, moe::kFp8>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
   }
-  if (dtype == MOE_DT_BF16) return launch_gemm_pair<S1, moe::kBf16>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  if (dtype == MOE_DT_BF16) return launch_gemm_pair<BN, S1, moe::kBf16>(ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  return MOE_ERR_INVALID_ARG;
+}
+
+template <bool S1>
+moe_status_t launch_gemm_pair_kind(int dtype, int bm, const CUtensorMap& ta, const CUtensorMap& tb,
+                                   const CUtensorMap& tb8, const CUtensorMap& tsfa, const CUtensorMap& tsfb,
+                                   const moe::GemmArgs& g, int max_pair_tiles, cudaStream_t s) {
+  if (bm == 16) return launch_gemm_pair_bn<16, S1>(dtype, ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
+  if (bm == 128) return launch_gemm_pair_bn<128, S1>(dtype, ta, tb, tb8, tsfa, tsfb, g, max_pair_tiles, s);
   return MOE_ERR_INVALID_ARG;
 }
 
@@ -732,7 +743,7 @@ moe_status_t moe_stage1_gemm(int dtype, const void* x, const void* x_scale, cons
     MOE_CK(cudaGetLastError());
   }
   const int max_tiles = cap_blocks * g.n_mt;
-  if (pair) return launch_gemm_pair_kind<true>(dtype, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
+  if (pair) return launch_gemm_pair_kind<true>(dtype, block_m, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
   return launch_gemm_kind<true>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
@@ -819,7 +830,7 @@ moe_status_t moe_stage2_gemm_accumulate(int dtype, const void* h, const void* h_
   g.counters = acc_ws ? reinterpret_cast<int*>(static_cast<float*>(acc_ws) + static_cast<size_t>(T) * H) : nullptr;
   g.out = static_cast<__nv_bfloat16*>(out);
   const int max_tiles = cap_blocks * g.n_mt;
-  if (pair) return launch_gemm_pair_kind<false>(dtype, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
+  if (pair) return launch_gemm_pair_kind<false>(dtype, block_m, ta, tb, tb16, tsfa, tsfb, g, max_tiles / 2, s);
   return launch_gemm_kind<false>(dtype, block_m, ta, tb, tb16, g, max_tiles, s);
 }
 
