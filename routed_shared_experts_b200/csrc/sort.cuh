@@ -25,9 +25,11 @@ struct SortArgs {
   int32_t* num_padded;    // [1]
 };
 
-// Shared memory of either kernel: tot[E], base[E], warp_cnt[32][E], warp sums [32].
+// Shared memory of either kernel: tot[E] (this CTA's counts), seg_cnt[E] and
+// seg_start[E] (every expert's count and padded segment start),
+// warp_cnt[32][E], warp sums [32].
 __host__ __device__ constexpr size_t sort_smem_bytes(int E) {
-  return (2 * static_cast<size_t>(E) + 32 * static_cast<size_t>(E) + 32) * sizeof(int);
+  return (3 * static_cast<size_t>(E) + 32 * static_cast<size_t>(E) + 32) * sizeof(int);
 }
 
 // Each warp owns one contiguous range [f0, f1) of the flat slots, so that a
@@ -142,7 +144,7 @@ __device__ __forceinline__ int sort_segment_prefix(int my_pad, int* wsum) {
   return incl - my_pad + wsum[warp];
 }
 
-// Expert tid's outputs: count, offset, block owners, sentinel padding.
+// Expert tid's count and offset (and, for the last expert, the total).
 __device__ __forceinline__ void sort_write_segment(const SortArgs& a, int e, int cnt, int excl, int pad) {
   a.counts[e] = cnt;
   a.offsets[e] = excl;
@@ -150,15 +152,33 @@ __device__ __forceinline__ void sort_write_segment(const SortArgs& a, int e, int
     a.offsets[a.E] = excl + pad;
     *a.num_padded = excl + pad;
   }
-  for (int b = excl / a.bm; b < (excl + pad) / a.bm; ++b) a.block_expert[b] = e;
-  for (int p = excl + cnt; p < excl + pad; ++p) a.sorted[p] = a.N;  // sentinel
+}
+
+// Block owners and sentinel padding of every expert, from seg_cnt / seg_start
+// in shared memory. The parts x 32 warps (every warp of every CTA taking part)
+// share the experts: warp w of part r takes experts e = 32 r + w, then every
+// (32 parts)-th after it, its lanes writing consecutive positions. (A segment
+// has up to bm - 1 padding slots; one thread per expert would issue them as
+// that many scattered stores, one after another.)
+__device__ __forceinline__ void sort_fill_padding(const SortArgs& a, const int* seg_cnt, const int* seg_start,
+                                                  int part, int parts) {
+  const int lane = threadIdx.x & 31;
+  const int gw = part * 32 + (threadIdx.x >> 5);
+  for (int e = gw; e < a.E; e += parts * 32) {
+    const int start = seg_start[e], cnt = seg_cnt[e];
+    const int end = start + (cnt + a.bm - 1) / a.bm * a.bm;
+    for (int b = start / a.bm + lane; b < end / a.bm; b += 32) a.block_expert[b] = e;
+    for (int p = start + cnt + lane; p < end; p += 32) a.sorted[p] = a.N;  // sentinel
+  }
 }
 
 // One CTA: warp w owns chunk w of 32 equal chunks of the slots.
 __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   extern __shared__ int ssm[];
   const int E = a.E;
-  int* warp_cnt = ssm + 2 * E;
+  int* seg_cnt = ssm + E;
+  int* seg_start = seg_cnt + E;
+  int* warp_cnt = seg_start + E;
   int* wsum = warp_cnt + 32 * E;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -176,9 +196,12 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   const int excl = sort_segment_prefix(pad, wsum);
   if (tid < E) {
     sort_write_segment(a, tid, cnt, excl, pad);
+    seg_cnt[tid] = cnt;
+    seg_start[tid] = excl;
     for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += excl;  // absolute start of warp w's slots of tid
   }
   __syncthreads();
+  sort_fill_padding(a, seg_cnt, seg_start, 0, 1);
   sort_place<1>(a, f0, f1, my_cnt_row);
 }
 
@@ -187,7 +210,8 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
 // cluster barrier makes every CTA's per-expert totals readable over
 // distributed shared memory; each CTA adds up, per expert, the totals of all
 // CTAs (the segment sizes, identical in every CTA) and of the CTAs before it
-// (its start inside the segment). CTA 0 writes the segment outputs. A second
+// (its start inside the segment). CTA 0 writes the counts and offsets; the
+// padding of the segments is spread over the warps of all CTAs. A second
 // cluster barrier, arrived at once the totals are read and waited on at the
 // end, keeps every CTA's shared memory alive until the others have read it.
 __global__ void __cluster_dims__(kSortCluster, 1, 1) __launch_bounds__(kSortThreads)
@@ -195,7 +219,9 @@ __global__ void __cluster_dims__(kSortCluster, 1, 1) __launch_bounds__(kSortThre
   extern __shared__ int ssm[];
   const int E = a.E;
   int* tot = ssm;  // this CTA's count of each expert, read by the cluster
-  int* warp_cnt = ssm + 2 * E;
+  int* seg_cnt = ssm + E;
+  int* seg_start = seg_cnt + E;
+  int* warp_cnt = seg_start + E;
   int* wsum = warp_cnt + 32 * E;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -233,10 +259,13 @@ __global__ void __cluster_dims__(kSortCluster, 1, 1) __launch_bounds__(kSortThre
   const int excl = sort_segment_prefix(pad, wsum);
   if (tid < E) {
     if (rank == 0) sort_write_segment(a, tid, cnt, excl, pad);
+    seg_cnt[tid] = cnt;
+    seg_start[tid] = excl;
     const int start = excl + before;
     for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += start;
   }
   __syncthreads();
+  sort_fill_padding(a, seg_cnt, seg_start, rank, kSortCluster);
   sort_place<kSortClusterBatch>(a, f0, f1, my_cnt_row);
   cluster_wait_acquire();  // no CTA leaves while another may still read its totals
 }
