@@ -154,6 +154,15 @@ __device__ __forceinline__ void sort_write_segment(const SortArgs& a, int e, int
   }
 }
 
+// Block owners and sentinel padding of one expert, by one thread: the
+// single-CTA sort's way at token blocks of up to 32 (at most 31 padding
+// slots), where it measured faster than sort_fill_padding (decode layer
+// sort 6.6 -> 4.7 us).
+__device__ __forceinline__ void sort_fill_expert(const SortArgs& a, int e, int cnt, int excl, int pad) {
+  for (int b = excl / a.bm; b < (excl + pad) / a.bm; ++b) a.block_expert[b] = e;
+  for (int p = excl + cnt; p < excl + pad; ++p) a.sorted[p] = a.N;  // sentinel
+}
+
 // Block owners and sentinel padding of every expert, from seg_cnt / seg_start
 // in shared memory. The parts x 32 warps (every warp of every CTA taking part)
 // share the experts: warp w of part r takes experts e = 32 r + w, then every
@@ -194,14 +203,16 @@ __global__ void __launch_bounds__(kSortThreads) k_align_sort(const SortArgs a) {
   const int cnt = sort_warp_prefix(warp_cnt, E);
   const int pad = tid < E ? (cnt + a.bm - 1) / a.bm * a.bm : 0;
   const int excl = sort_segment_prefix(pad, wsum);
+  const bool per_thread_pad = a.bm <= 32;
   if (tid < E) {
     sort_write_segment(a, tid, cnt, excl, pad);
+    if (per_thread_pad) sort_fill_expert(a, tid, cnt, excl, pad);
     seg_cnt[tid] = cnt;
     seg_start[tid] = excl;
     for (int w = 0; w < 32; ++w) warp_cnt[w * E + tid] += excl;  // absolute start of warp w's slots of tid
   }
   __syncthreads();
-  sort_fill_padding(a, seg_cnt, seg_start, 0, 1);
+  if (!per_thread_pad) sort_fill_padding(a, seg_cnt, seg_start, 0, 1);
   sort_place<1>(a, f0, f1, my_cnt_row);
 }
 
