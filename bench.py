@@ -30,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import time
@@ -109,12 +110,21 @@ def tensor_peak(dtype: str):
 GEMM_SOURCES = ("gemm.cuh", "ptx.cuh", "moe_b200.cu")  # the GEMM kernels and the launcher that picks their instances
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank lines: what the compiler sees."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def src_hash() -> str:
+    """Hash of the GEMM kernels' code (comments left out, so that a counter
+    taken on a kernel stays valid across edits of its comments only)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "routed_shared_experts_b200", "csrc")
     for f in GEMM_SOURCES:
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -3,16 +3,20 @@
 // Stage 1 (gate_up + SiLU-and-mul) and stage 2 (down + weighted scatter-reduce
 // + shared-expert addend) share one persistent, warp-specialised kernel:
 //
-//   warp 0      TMA producer: weight tile (128 rows x 128 K-bytes) and token
-//               tile (BN rows x 128 K-bytes) per pipeline stage. Stage-1 token
-//               rows come from a copy of x in sorted order (k_stage1_prep).
-//               MXFP8 adds the stage's two 512-byte scale tiles.
+//   warp 0      TMA producer: per pipeline stage, the weight tile (128 rows
+//               x 128 K-bytes per K atom; two atoms per stage up to 128-token
+//               tiles) and, with one producer warp, the token tile (BN rows x
+//               the same K-bytes). Stage-1 token rows come from a copy of x in
+//               sorted order (k_stage1_prep). Block-scaled kernels add the
+//               stage's 512-byte scale tiles.
+//   warp 2      second producer (64+-token tiles, block-scaled kernels): the
+//               token tile and its scale tiles, warp 0 keeping the weights'.
 //   warp 1      TMEM allocator + MMA issuer (one thread): tcgen05.mma with the
 //               weights as A (M = 128) and the tokens as B (N = BN), fp32
-//               accumulator in TMEM, a ring of 2 or 4 across tiles. MXFP8
-//               copies the scale tiles into TMEM (tcgen05.cp) and issues the
-//               block-scaled MMA.
-//   warps 2..   epilogue, one or two warpgroups taking alternate tiles:
+//               accumulator in TMEM, a ring of 2 to 4 across tiles.
+//   warp 3      block-scaled kernels: copies each stage's scale tiles into
+//               TMEM (tcgen05.cp) for the block-scaled MMA.
+//   then        epilogue, one or two warpgroups taking alternate tiles:
 //               tcgen05.ld of the accumulator, then
 //               stage 1: operand scales, SiLU(gate) * up, store h in the
 //               stage-2 operand format (bf16, e4m3 with a per-row scale, or
@@ -37,7 +41,7 @@
 namespace moe {
 
 constexpr int kTileM = 128;       // weight rows per tile = MMA M
-constexpr int kTileKBytes = 128;  // K bytes per pipeline stage = one 128-byte swizzle row
+constexpr int kTileKBytes = 128;  // K bytes of one K atom = one 128-byte swizzle row
 constexpr int kEpiThreads = 128;  // one epilogue warpgroup
 constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
 constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)

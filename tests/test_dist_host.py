@@ -121,3 +121,17 @@ def test_weight_copies_put_every_step_over_three_l2s():
         assert n == 1 or (n - 1) * step < 3 * bench.L2_BYTES
         assert "come from HBM" in bench.l2_note(step, n)
     assert bench.weight_copies(0.81e9) == 1 and bench.weight_copies(1.8e6) == 210
+
+
+def test_traffic_records_follow_the_kernel_code_not_its_comments():
+    sys.path.insert(0, ROOT)
+    import bench
+    src = "// a comment\nint f(int x) { /* inline\n block */ return x + 1; }  // trailing\n\n"
+    assert bench._code_only(src) == "int f(int x) {  return x + 1; }"
+    edited = src.replace("a comment", "another comment").replace("trailing", "tail")
+    assert bench._code_only(edited) == bench._code_only(src)
+    assert bench._code_only(src.replace("x + 1", "x + 2")) != bench._code_only(src)
+    # every recorded figure is keyed to a hash of that form, and looked up by it
+    import json
+    rows = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")))
+    assert rows and all(len(r["src_sha"]) == 16 and r["dram_bytes_per_launch"] > 0 for r in rows)
