@@ -44,7 +44,7 @@ constexpr int kTileM = 128;       // weight rows per tile = MMA M
 constexpr int kTileKBytes = 128;  // K bytes of one K atom = one 128-byte swizzle row
 constexpr int kEpiThreads = 128;  // one epilogue warpgroup
 constexpr int kSfTile = 512;      // bytes of one MXFP8 scale tile (128 rows x 4 K blocks)
-constexpr int kSfSlots = 4;       // TMEM ring of scale tiles (8 columns each: A then B)
+constexpr int kSfSlots = 4;       // pairs: TMEM ring of scale tiles (8 columns per K atom: A then B)
 constexpr int kFinBatch = 8;      // stage-2 finalisation: token columns per batch of loads
 // kMx4: MXFP4 weights (e2m1, two per byte in memory; the tensor map unpacks
 // each 16-element group into 16 bytes of shared memory, so a weight tile has
@@ -150,7 +150,7 @@ struct GemmSmem {
   static constexpr int kBarOffset = STAGES * kStageBytes;
   // scale tiles in TMEM: copied by warp 3 into slot `stage` (one-CTA tiles;
   // 8 columns per atom: the A tiles, then the B tiles), else by the MMA
-  // thread into a ring of kSfSlots (pairs, one atom per stage; warp 3 idles)
+  // thread into a ring of kSfSlots (pairs; warp 3 idles)
   static constexpr bool kSfWarp = EpiCfg<BN, KIND, S1>::kSfWarp && !PAIR;
   static constexpr int kSfRing = kSfWarp ? STAGES : kSfSlots;
   // full[S], empty[S], acc_full[A], acc_empty[A], drain, then sf_full[S] with the scale-copy warp
