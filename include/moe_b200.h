@@ -144,8 +144,8 @@ size_t moe_stage2_workspace_bytes(int T, int H);
  *  - MOE_DT_FP8_E4M3: the unquantised h as fp32 [rows, I], a per-tile row
  *    amax and one arrival counter per token block;
  *  - the token rows of x copied into sorted order [rows, H] (x's element
- *    type), which the GEMM then reads with one TMA box per stage (identity
- *    routing reads x itself and leaves this part unused);
+ *    type), which the GEMM then reads with one TMA box per 128-byte K atom
+ *    (identity routing reads x itself and leaves this part unused);
  *  - MOE_DT_MXFP8_E4M3 / MOE_DT_MXFP4_E2M1: the token scale bytes placed in
  *    512-byte tiles, one per (token block, 128 columns of H).
  * The caller zeroes it ONCE after allocating it; each complete call leaves the
@@ -293,7 +293,7 @@ moe_status_t moe_quantize_activations(int dtype, const void* x, int T, int H, vo
  * then h_r is stored in the stage-2 operand format ([6106]: quantisation fused
  * after the activation). tcgen05 tensor cores, weights streamed by TMA; token
  * rows (and MXFP8 token scales) copied into sorted order by a preparation
- * kernel launched first on `stream`, then read one box per stage. The
+ * kernel launched first on `stream`, then read one box per 128-byte K atom. The
  * preparation kernel records device error 3 for a sorted slot id that is
  * neither a slot nor the padding value T*top_k.
  *   dtype      MOE_DT_BF16, MOE_DT_FP8_E4M3, MOE_DT_MXFP8_E4M3 or
